@@ -1,0 +1,420 @@
+"""Benchmark of the Medusa verify step (heads + top-s, tree expansion, tree
+attention, acceptance, KV compaction) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+                    [--impl ours|reference]
+
+One process per GPU (torchrun for N > 1).  Every rank runs its own replica
+of the step on its own sequences (data parallel, no collective on the data
+path: weak scaling).  Rank 0 prints one JSON line.  `--impl reference` times
+the plain fp64 CPU oracle on sampled slices of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from medusa_head_speculative_02_b200.synthetic import CONFIGS, gen_inputs  # noqa: E402
+
+DEFAULT_CONFIG = "7b_b1"
+METRIC = "verify steps/s"
+
+
+# ---------------------------------------------------------------------------- helpers
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank float over the process group (identity without one)."""
+    if not torch.distributed.is_available() or not torch.distributed.is_initialized():
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(units_per_rank: float, seconds_per_rank: float, world: int, device) -> dict:
+    """Whole-job throughput: units all ranks processed / max time over ranks."""
+    t = max_over_ranks(seconds_per_rank, device)
+    return {"seconds": t, "value": units_per_rank * world / t if t > 0 else 0.0}
+
+
+def barrier():
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.barrier()
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons of this rank's GPU while running."""
+
+    FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.bus = None
+        try:
+            p = torch.cuda.get_device_properties(device_index)
+            self.bus = "%08X:%02X:%02X.0" % (getattr(p, "pci_domain_id", 0),
+                                              getattr(p, "pci_bus_id", 0),
+                                              getattr(p, "pci_device_id", 0))
+        except Exception:
+            pass
+        self.rows, self.proc, self.thread = [], None, None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([c.strip() for c in line.split(",")])
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+        rows = [r for r in self.rows if len(r) >= 10]
+        if self.bus:
+            mine = [r for r in rows if r[1].upper().endswith(self.bus[-7:])]
+            rows = mine or rows
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        reasons = set()
+        for r in rows:
+            for name, v in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                                "sw_power_cap"), r[6:10]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": d.get("hbm_gbs", 6650.0), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "src": "fallback"}
+
+
+# ---------------------------------------------------------------------------- oracle sampler
+class OracleSampler:
+    """Times the fp64 CPU oracle on bounded slices of one verify step and
+    scales each slice by its share of the step (units of that operation)."""
+
+    def __init__(self, cfg, x, vlogits, target_ms: float):
+        from oracle import medusa_oracle as O
+        self.O, self.cfg = O, cfg
+        self.x = {k: v.cpu() for k, v in x.items()}
+        self.vlog = vlogits.cpu()
+        self.plan = O.tree_plan(cfg.K, cfg.s, cfg.N)
+        g = torch.Generator().manual_seed(1)
+        self.topk = torch.stack([torch.randperm(cfg.V, generator=g)[:cfg.K * cfg.s]
+                                 .view(cfg.K, cfg.s) for _ in range(cfg.B)])
+        self.tok, _ = O.build_tree(self.plan, self.x["root_tok"], self.topk, self.x["prefix_len"])
+        self.u = O.heads_hidden(self.x["h"], self.x["W1"], self.x["b1"], 0, rows=None)
+        # (name, full units, slice units); slices sized by a calibration pass
+        self.ops = {"stage1": [cfg.K * cfg.d, 64], "stage2": [cfg.K * cfg.V, 512],
+                    "topk": [cfg.B * cfg.K, 1], "tree": [1, 1],
+                    "attention": [cfg.B * cfg.N * cfg.Hq, 16], "accept": [cfg.B, 1],
+                    "compact": [cfg.B, 1]}
+        self.times = {k: [] for k in self.ops}
+        self.names = list(self.ops)
+        self.j = 0
+        self._calibrate(target_ms / 1000.0)
+
+    def _run(self, name, n):
+        O, c, x = self.O, self.cfg, self.x
+        j = self.j
+        if name == "stage1":
+            k = j % c.K
+            lo = (j * n) % c.d
+            O.heads_hidden(x["h"], x["W1"], x["b1"], k, rows=np.arange(lo, min(c.d, lo + n)))
+        elif name == "stage2":
+            k = j % c.K
+            lo = (j * n) % c.V
+            O.heads_logits(self.u, x["W2"], k, vocab=np.arange(lo, min(c.V, lo + n)))
+        elif name == "topk":
+            # one (sequence, head) row of V logits; any length-V row costs the same
+            O.topk_row(self.vlog[j % c.B, 0], c.s)
+        elif name == "tree":
+            O.build_tree(self.plan, x["root_tok"], self.topk, x["prefix_len"])
+        elif name == "attention":
+            rows = [((j + r) % c.B, ((j + r) // c.B) % c.N, (j * 7 + r) % c.Hq) for r in range(n)]
+            O.tree_attention(x["q"], x["k_cache"], x["v_cache"], x["prefix_len"], self.plan,
+                             1.0 / np.sqrt(c.dh), rows=rows)
+        elif name == "accept":
+            b = j % c.B
+            if c.accept in ("greedy", "both"):
+                O.accept_greedy(self.vlog[b:b + 1], self.tok[b:b + 1], self.plan)
+            if c.accept in ("typical", "both"):
+                O.accept_typical(self.vlog[b:b + 1], self.tok[b:b + 1], self.plan, c.temperature,
+                                 c.eps, c.delta)
+        elif name == "compact":
+            b = j % c.B
+            O.kv_compact(x["k_cache"][b:b + 1], x["v_cache"][b:b + 1], x["prefix_len"][b:b + 1],
+                         torch.tensor([2]), torch.tensor([[0, 1, 2] + [-1] * (c.K - 2)]))
+
+    def _calibrate(self, target_s):
+        for name, (full, n) in self.ops.items():
+            t0 = time.perf_counter()
+            self._run(name, n)
+            dt = time.perf_counter() - t0
+            if name in ("stage1", "stage2", "attention") and dt > 0:
+                n2 = int(max(1, min(full, n * target_s / dt)))
+                self.ops[name][1] = n2
+
+    def step(self):
+        name = self.names[self.j % len(self.names)]
+        full, n = self.ops[name]
+        t0 = time.perf_counter()
+        self._run(name, n)
+        self.times[name].append((time.perf_counter() - t0) * full / n)
+        self.j += 1
+
+    def estimate_step_seconds(self) -> float:
+        return sum(statistics.mean(v) for v in self.times.values() if v)
+
+    def sample_desc(self) -> str:
+        d = {k: f"{v[1]}/{v[0]}" for k, v in self.ops.items()}
+        return ("per step one op slice, round robin; slice/full units: " +
+                ", ".join(f"{k} {v}" for k, v in d.items()) +
+                "; each op's mean slice time scaled by full/slice units and summed")
+
+
+# ---------------------------------------------------------------------------- arms
+def run_reference(args, cfg, world, rank):
+    if rank != 0:
+        return 0
+    t_setup = time.time()
+    x = gen_inputs(cfg, "cpu", seed=0)
+    from oracle import medusa_oracle as O
+    plan = O.tree_plan(cfg.K, cfg.s, cfg.N)
+    from medusa_head_speculative_02_b200.synthetic import plant_verify_logits
+    g = torch.Generator().manual_seed(1)
+    topk = torch.stack([torch.randperm(cfg.V, generator=g)[:cfg.K * cfg.s].view(cfg.K, cfg.s)
+                        for _ in range(cfg.B)])
+    tok, _ = O.build_tree(plan, x["root_tok"], topk, x["prefix_len"])
+    vlog = plant_verify_logits(cfg, plan["parent"], tok, "cpu", 0)
+    budget_s = float(os.environ.get("MEDUSA_REF_BUDGET_S", "150"))
+    target_ms = max(2.0, min(40.0, 1000.0 * budget_s / max(1, args.steps + args.warmup)))
+    S = OracleSampler(cfg, x, vlog, target_ms)
+    for _ in range(args.warmup):
+        S.step()
+    S.times = {k: [] for k in S.ops}
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        S.step()
+    wall = time.perf_counter() - t0
+    est = S.estimate_step_seconds()
+    value = 1.0 / est if est > 0 else 0.0
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": est * 1000.0, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "batch": cfg.B, "d": cfg.d, "vocab": cfg.V,
+                       "heads": cfg.K, "top_s": cfg.s, "tree_nodes": cfg.N, "q_heads": cfg.Hq,
+                       "kv_heads": cfg.Hkv, "head_dim": cfg.dh, "prefix": [cfg.L_lo, cfg.L_hi],
+                       "accept": cfg.accept},
+            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores, "kind": "oracle",
+                             "sample": S.sample_desc(), "wall_s": wall,
+                             "setup_s": t0 - t_setup},
+            "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, cfg, world, rank, local):
+    from medusa_head_speculative_02_b200.step import HostIO, VerifyStep
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    st = VerifyStep(cfg, dev, seed=rank)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        st.run()
+    torch.cuda.synchronize(dev)
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for k in range(K):
+        e = ev[k]
+        e[0].record(stream)
+        st.heads()
+        e[1].record(stream)
+        st.build_tree()
+        e[2].record(stream)
+        st.attention()
+        e[3].record(stream)
+        st.accept()
+        st.compact()
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    elapsed_s = start.elapsed_time(end) / 1000.0
+    heads_ms = statistics.mean(ev[k][0].elapsed_time(ev[k][1]) for k in range(K))
+    attn_ms = statistics.mean(ev[k][2].elapsed_time(ev[k][3]) for k in range(K))
+    agg = aggregate(K, elapsed_s, world, dev)
+    ms_per_step = agg["seconds"] * 1000.0 / K
+    alen = st.accept_len.float().mean().item()
+
+    # end to end through the public API with host buffers
+    io = HostIO(st)
+    Ke = max(10, K // 8)
+    for _ in range(3):
+        io.step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(Ke):
+        io.step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e = aggregate(Ke, e0.elapsed_time(e1) / 1000.0, world, dev)
+
+    peaks = measured_peaks()
+    hb = st.heads_bytes()
+    ab = st.attention_bytes()
+    heads_gbs = hb / (heads_ms / 1000.0) / 1e9
+    attn_gbs = ab / (attn_ms / 1000.0) / 1e9
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "heads_traffic.json")
+    if os.path.exists(tpath):
+        try:
+            traffic = json.load(open(tpath)).get(cfg.name)
+        except Exception:
+            traffic = None
+
+    line = None
+    if rank == 0:
+        line = {"metric": METRIC, "value": agg["value"], "unit": "steps/s", "n_gpus": world,
+                "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16" if cfg.dtype == "bf16" else "f32", "data": "synthetic",
+                "config": {"workload": cfg.name, "batch": cfg.B, "d": cfg.d, "vocab": cfg.V,
+                           "heads": cfg.K, "top_s": cfg.s, "tree_nodes": cfg.N,
+                           "q_heads": cfg.Hq, "kv_heads": cfg.Hkv, "head_dim": cfg.dh,
+                           "prefix": [cfg.L_lo, cfg.L_hi], "accept": cfg.accept,
+                           "parallelism": f"dp{world} (independent replicas)",
+                           "l2": "inputs larger than L2: each step streams "
+                                 f"{hb / 1e9:.2f} GB of head weights, evicting the "
+                                 f"{ab / 1e6:.1f} MB attention working set"},
+                "tokens_per_s": agg["value"] * cfg.B * (1.0 + alen),
+                "mean_accept_len": alen,
+                "roofline": {"kernel": "medusa_heads_forward (two heads_tc_kernel GEMMs + "
+                                       "top-s merge)",
+                             "bound": "hbm", "achieved": heads_gbs, "peak": peaks["hbm_gbs"],
+                             "unit": "GB/s", "frac": heads_gbs / peaks["hbm_gbs"],
+                             "traffic": traffic, "peak_src": peaks["src"],
+                             "algorithmic_bytes": hb, "avg_ms": heads_ms},
+                "kernels": {"tree_attention": {"achieved": attn_gbs, "unit": "GB/s",
+                                               "frac": attn_gbs / peaks["hbm_gbs"],
+                                               "algorithmic_bytes": ab, "avg_ms": attn_ms}},
+                "e2e": {"value": e2e["value"], "unit": "steps/s",
+                        "h2d_bytes_per_step": io.h2d_bytes(),
+                        "d2h_bytes_per_step": io.d2h_bytes(), "steps": Ke},
+                "gpu_launches": st.launches_per_step() * K,
+                "clocks": clk}
+    # CPU baseline: the oracle on rank 0 at N = 1 only
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        S = OracleSampler(cfg, st.x, st.vlogits, target_ms=40.0)
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < args.cpu_seconds:
+            S.step()
+        est = S.estimate_step_seconds()
+        line["cpu_baseline"] = {"value": 1.0 / est if est > 0 else 0.0, "unit": "steps/s",
+                                "cores": blas_threads(), "kind": "oracle",
+                                "sample": S.sample_desc(),
+                                "host_cores_available": cpu_cores()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=list(CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = CONFIGS[args.config]
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, cfg, world, rank)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    try:
+        return run_ours(args, cfg, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

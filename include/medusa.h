@@ -1,0 +1,235 @@
+/*
+ * medusa.h - C ABI of libmedusa.so: the per-step Medusa draft-and-verify
+ * chain (heads -> top-s -> tree -> tree attention -> acceptance -> KV
+ * compaction) as CUDA kernels for sm_100a (B200).
+ *
+ * Sources (page title, then section):
+ *   [MD] "論文解説: Medusa — 複数デコーディングヘッドによるLLM推論高速化フレームワーク":
+ *        "Medusa Headのアーキテクチャ" (head equation), "ツリーアテンションによる
+ *        並列検証" (top-s, Cartesian-product tree, ancestor mask),
+ *        "候補選択：Typical Acceptance" (typical and greedy acceptance).
+ *   [EX] "メドゥーサ デコーディング ヘッド", "ディープダイブ" (accept the longest
+ *        matching prefix).
+ *   [FR] "Medusa" (glossaire), "Attention en arbre" (each node sees only its
+ *        ancestors; the longest valid path is accepted).
+ *
+ * Conventions shared by every call:
+ *   - Return value: MEDUSA_OK (0) or a negative medusa_status.  On error
+ *     medusa_last_error() (thread-local) describes the failure.  Nothing is
+ *     launched when argument validation fails.  No C++ exception crosses
+ *     the ABI.
+ *   - Tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or retains them.  Layouts are row-major and
+ *     contiguous as written in brackets, e.g. h [B][d].
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every compute call is asynchronous on that stream and never
+ *     synchronizes the host.
+ *   - `ws`/`ws_bytes` is caller-owned device scratch of at least the size the
+ *     matching *_workspace_size() call returns, 256-byte aligned.  Its
+ *     contents on entry are irrelevant; calls sharing one workspace must be
+ *     ordered on the GPU (same stream, or synchronized).
+ *   - Outputs are completely overwritten; no pre-zeroing is required.
+ *   - dtype is MEDUSA_F32 or MEDUSA_BF16 and applies to every floating-point
+ *     tensor argument of the call that is not explicitly typed float*.
+ *   - Device-side waits are bounded.  A kernel whose wait runs out sets a
+ *     device status word and returns early (its outputs are then undefined);
+ *     medusa_device_status() reports MEDUSA_ERR_TIMEOUT.
+ */
+#ifndef MEDUSA_H_
+#define MEDUSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MEDUSA_OK = 0,
+  MEDUSA_ERR_INVALID_ARG = -1, /* null pointer, bad size, bad tree, ... */
+  MEDUSA_ERR_UNSUPPORTED = -2, /* valid but not implemented (dtype/shape) */
+  MEDUSA_ERR_CUDA = -3,        /* a CUDA runtime/driver call failed */
+  MEDUSA_ERR_TIMEOUT = -4      /* a device-side bounded wait ran out */
+} medusa_status;
+
+typedef enum { MEDUSA_F32 = 0, MEDUSA_BF16 = 1 } medusa_dtype;
+
+/* Opaque, immutable tree plan (library-owned host + device copy). */
+typedef struct medusa_tree medusa_tree_t;
+
+/* Limits of this build. */
+#define MEDUSA_MAX_K 8      /* Medusa heads = maximum tree depth */
+#define MEDUSA_MAX_S 16     /* top-s per head */
+#define MEDUSA_MAX_N 256    /* tree nodes, root included */
+
+/* Thread-local message for the last failing call on this thread ("" if none). */
+const char* medusa_last_error(void);
+
+/* Library version string. */
+const char* medusa_version(void);
+
+/*
+ * Reads (and with clear != 0 resets) the device status word of the current
+ * device.  Synchronizes the device.  *status receives MEDUSA_OK or
+ * MEDUSA_ERR_TIMEOUT.  Returns MEDUSA_ERR_CUDA if the device is unusable.
+ */
+int medusa_device_status(int* status, int clear);
+
+/* ------------------------------------------------------------------------
+ * Tree plan.  [MD] "ツリーアテンションによる並列検証": each of the K heads
+ * proposes its top-s tokens; their Cartesian product is pruned to a tree.
+ * Pruning rule: keep the N rank tuples (r_1..r_D), 0 <= D <= K, 0-based
+ * ranks, with the largest score prod_i 0.5^{r_i} * 0.8^D.  N includes the
+ * root (the empty tuple).  Score ties break by (depth asc, tuple
+ * lexicographic asc).  Node order is (depth asc, tuple lexicographic asc):
+ * node 0 is the root and parent[n] < n.
+ * ------------------------------------------------------------------------ */
+
+/*
+ * Host only (no CUDA call): fills caller-owned HOST arrays
+ *   parent[N] (-1 for the root), depth[N], rank_path[N][K] (-1 padded),
+ *   anc_mask[N][(N+31)/32] (bit j of row i set iff node j is node i or one
+ *   of its ancestors).
+ * Any output pointer may be NULL.  Errors: INVALID_ARG if K, s, N are out of
+ * [1, MEDUSA_MAX_*] or N exceeds the number of tuples 1 + s + ... + s^K.
+ */
+int medusa_tree_plan_host(int K, int s, int N, int32_t* parent, int32_t* depth,
+                          int32_t* rank_path, uint32_t* anc_mask);
+
+/*
+ * Builds the plan and uploads it to the CURRENT device (synchronous upload).
+ * *out receives the handle; release it with medusa_tree_destroy.
+ */
+int medusa_tree_create(int K, int s, int N, medusa_tree_t** out);
+int medusa_tree_destroy(medusa_tree_t* tree);
+
+/* Host copies of a plan's shape and arrays (same layouts as plan_host). */
+int medusa_tree_info(const medusa_tree_t* tree, int* K, int* s, int* N,
+                     int32_t* parent, int32_t* depth, int32_t* rank_path,
+                     uint32_t* anc_mask);
+
+/* ------------------------------------------------------------------------
+ * Medusa heads.  [MD] "Medusa Headのアーキテクチャ":
+ *   logits_k[b] = W2_k (SiLU(W1_k h[b] + b1_k) + h[b]),  k = 0..K-1,
+ * SiLU(x) = x * sigmoid(x).  Head k (0-based) predicts the token k+2 steps
+ * ahead of the last verified token.
+ * ------------------------------------------------------------------------ */
+
+/* Scratch bytes needed by medusa_heads_forward for these sizes. */
+size_t medusa_heads_workspace_size(int B, int d, int V, int K, int s, int dtype);
+
+/*
+ * h [B][d]; W1 [K][d][d] (row = output feature); b1 [K][d] or NULL (= 0);
+ * W2 [K][V][d] (row = vocabulary entry); all of `dtype`.
+ * Outputs (each may be NULL, not both):
+ *   logits   [B][K][V] fp32;
+ *   topk_idx [B][K][s] int32: the s best vocabulary ids of each (b, k),
+ *            by logit descending, ties to the lower id;
+ *   topk_val [B][K][s] fp32 (only written when topk_idx is non-NULL).
+ * bf16: W1 and W2 are streamed by tcgen05 tensor-core GEMMs (TMA-fed, fp32
+ * accumulation in TMEM) with the bias, SiLU and residual fused in the first
+ * GEMM's epilogue and a partial top-s fused in the second's.  The hidden
+ * activation u is passed to the second GEMM as a bf16 hi/lo pair (u = hi +
+ * lo), so it keeps ~16 mantissa bits.  fp32: SIMT kernels.
+ * Limits: d % 8 == 0; B <= 32 (bf16) or 16 (fp32); K <= MEDUSA_MAX_K;
+ * 1 <= s <= MEDUSA_MAX_S, s <= V.  Pointers 16-byte aligned.
+ */
+int medusa_heads_forward(const void* h, const void* W1, const void* b1,
+                         const void* W2, int B, int d, int V, int K, int dtype,
+                         float* logits, int s, int32_t* topk_idx,
+                         float* topk_val, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/*
+ * Top-s of each row of logits [R][V] (dtype): idx [R][s] int32 (value
+ * descending, ties to the lower index); val [R][s] fp32 or NULL.
+ * 1 <= s <= MEDUSA_MAX_S, s <= V.
+ */
+int medusa_topk(const void* logits, int dtype, int R, int V, int s,
+                int32_t* idx, float* val, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Tree expansion: node n with rank tuple (r_1..r_D) carries
+ *   tree_tok[b][n] = root_tok[b]                      if D == 0
+ *                  = topk_idx[b][D-1][r_D]            otherwise
+ * (head D-1, 0-based, proposes the token at tree depth D), and
+ *   tree_pos[b][n] = prefix_len[b] + D.
+ * root_tok [B], topk_idx [B][K][s], prefix_len [B] int32 device arrays.
+ * ------------------------------------------------------------------------ */
+int medusa_build_tree(const medusa_tree_t* tree, const int32_t* root_tok,
+                      const int32_t* topk_idx, const int32_t* prefix_len,
+                      int B, int32_t* tree_tok, int32_t* tree_pos,
+                      void* stream);
+
+/* ------------------------------------------------------------------------
+ * Tree attention.  [MD] Mask_ij = 1 iff j is an ancestor of i (the node
+ * itself included).  For sequence b, tree node i and query head h:
+ *   out[b][i][h] = softmax_j(scale * q[b][i][h] . k_j) v_j
+ * over the keys j in {prefix slots 0..L_b-1} U {slot L_b + a : a is node i
+ * or an ancestor of i}, where L_b = prefix_len[b] and the tree tokens' K/V
+ * sit at slots L_b..L_b+N-1 of the cache.  kv-head of query head h is
+ * h / (Hq/Hkv).
+ * q [B][N][Hq][dh]; k_cache, v_cache [B][Lcap][Hkv][dh]; out [B][N][Hq][dh].
+ * Requires L_b + N <= Lcap (checked on the device: rows of a sequence that
+ * violates it are written as zeros and the status word is left untouched),
+ * Hq % Hkv == 0, dh in {64, 128}.
+ * ------------------------------------------------------------------------ */
+size_t medusa_tree_attention_workspace_size(const medusa_tree_t* tree, int B,
+                                            int Hq, int Hkv, int dh, int Lcap);
+
+int medusa_tree_attention(const void* q, const void* k_cache,
+                          const void* v_cache, const int32_t* prefix_len,
+                          const medusa_tree_t* tree, int B, int Hq, int Hkv,
+                          int dh, int Lcap, float scale, int dtype, void* out,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Acceptance over verify logits vlogits [B][N][V] (dtype) for the tree
+ * tokens tree_tok [B][N].
+ *   greedy  ([MD], temperature 0): node n != 0 is accepted iff its parent is
+ *           accepted and argmax(vlogits[b][parent]) == tree_tok[b][n]
+ *           (argmax ties to the lowest id).
+ *   typical ([MD] "候補選択：Typical Acceptance"): node n != 0 is accepted iff
+ *           its parent is accepted and p(tok) > min(eps, delta*exp(-H(p)))
+ *           with p = softmax(vlogits[b][parent] / temperature) and
+ *           H(p) = -sum p ln p.
+ * The deepest accepted node wins (ties: lowest node index) ([EX], [FR]).
+ * Outputs: accept_len [B] (its depth, 0..K); accept_nodes [B][K+1] (node
+ * ids on the root-to-node path, root first, -1 padded); next_tok [B] (argmax
+ * of the winning node's verify row).
+ * ------------------------------------------------------------------------ */
+size_t medusa_accept_workspace_size(const medusa_tree_t* tree, int B, int V);
+
+int medusa_accept_greedy(const void* vlogits, int dtype, const int32_t* tree_tok,
+                         const medusa_tree_t* tree, int B, int V,
+                         int32_t* accept_len, int32_t* accept_nodes,
+                         int32_t* next_tok, void* ws, size_t ws_bytes,
+                         void* stream);
+
+int medusa_accept_typical(const void* vlogits, int dtype,
+                          const int32_t* tree_tok, const medusa_tree_t* tree,
+                          int B, int V, float temperature, float eps,
+                          float delta, int32_t* accept_len,
+                          int32_t* accept_nodes, int32_t* next_tok, void* ws,
+                          size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * KV compaction of the accepted path (the accepted tokens' K/V become the
+ * contiguous continuation of the sequence):
+ *   for j = 1..accept_len[b]: slot L_b + j <- slot L_b + accept_nodes[b][j]
+ * in k_cache and v_cache [B][Lcap][Hkv][dh] (in place, bit-exact), and
+ *   new_len[b] = L_b + 1 + accept_len[b]   (root + accepted tokens).
+ * accept_nodes [B][K+1] as written by the accept calls.  Entries with
+ * accept_len outside [0, K] or nodes outside the cache are skipped.
+ * ------------------------------------------------------------------------ */
+int medusa_kv_compact(void* k_cache, void* v_cache, const int32_t* prefix_len,
+                      const int32_t* accept_len, const int32_t* accept_nodes,
+                      int B, int Hkv, int dh, int Lcap, int K, int dtype,
+                      int32_t* new_len, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MEDUSA_H_ */

@@ -1,0 +1,290 @@
+// Acceptance of the verified tree.
+//
+// Medusa paper digest ("論文解説: Medusa"), section "候補選択：Typical
+// Acceptance": a candidate x is accepted iff p(x) > min(eps, delta *
+// exp(-H(p))), H(p) = -sum p log p; with temperature 0 the check is an argmax
+// comparison.  Explainer ("メドゥーサ デコーディング ヘッド", "ディープダイブ")
+// and glossary ("Medusa", "Attention en arbre"): the longest path whose
+// tokens are all valid is accepted.
+//
+// Phase 1 (row_reduce_kernel, HBM stream): every verify row [V] is split
+// into chunks; each CTA reduces its chunk to the 64-bit argmax key (value
+// desc, index asc) and, for typical acceptance, the base-2 online softmax
+// statistics of z = l * log2(e) / T:  m = max z, Z = sum 2^(z-m),
+// S = sum 2^(z-m) (z-m).  Natural-log entropy: H = ln Z - ln2 * S / Z.
+// Phase 2 (accept_walk_kernel, one warp per sequence): merge the chunks of
+// the N rows, decide every node's own condition against its parent row,
+// accept a node iff its whole root path satisfies the condition (ancestor
+// bitmask test), take the deepest accepted node (ties: lowest index) and
+// emit its path and the argmax of its row.
+#include "common.cuh"
+#include "internal.h"
+
+namespace medusa {
+namespace {
+
+constexpr int kRedThreads = 256;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct RowPart {
+  uint64_t key;
+  float m, Z, S, pad;
+};
+
+struct Soft {
+  float m, Z, S;
+};
+
+__device__ __forceinline__ void soft_add(Soft& a, float z) {
+  if (a.Z == 0.f) {
+    a.m = z;
+    a.Z = 1.f;
+    a.S = 0.f;
+  } else if (z <= a.m) {
+    const float t = z - a.m;
+    const float e = exp2f(t);
+    a.Z += e;
+    a.S = fmaf(e, t, a.S);
+  } else {
+    const float t = a.m - z;  // < 0
+    const float c = exp2f(t);
+    a.S = c * fmaf(t, a.Z, a.S);
+    a.Z = fmaf(c, a.Z, 1.f);
+    a.m = z;
+  }
+}
+
+__device__ __forceinline__ Soft soft_merge(Soft a, Soft b) {
+  if (b.Z == 0.f) return a;
+  if (a.Z == 0.f) return b;
+  const float M = fmaxf(a.m, b.m);
+  const float ta = a.m - M, tb = b.m - M;
+  const float ca = exp2f(ta), cb = exp2f(tb);
+  Soft r;
+  r.m = M;
+  r.Z = ca * a.Z + cb * b.Z;
+  r.S = ca * fmaf(ta, a.Z, a.S) + cb * fmaf(tb, b.Z, b.S);
+  return r;
+}
+
+template <typename T, bool TYPICAL>
+__global__ void __launch_bounds__(kRedThreads)
+    row_reduce_kernel(const T* __restrict__ vlog, int V, int chunk, int splits, float zscale,
+                      RowPart* __restrict__ parts) {
+  const size_t row = blockIdx.x;
+  const int sp = blockIdx.y;
+  const int lo = sp * chunk;
+  const int hi = min(V, lo + chunk);
+  const T* xr = vlog + row * (size_t)V;
+  uint64_t best = 0ull;
+  Soft sf{-INFINITY, 0.f, 0.f};
+  constexpr int VEC = 16 / sizeof(T);
+  const bool vec_ok = ((((uintptr_t)(xr + lo)) & 15u) == 0) && ((hi - lo) % VEC == 0);
+  if (vec_ok) {
+    const uint4* p = reinterpret_cast<const uint4*>(xr + lo);
+    const int nv = (hi - lo) / VEC;
+    for (int i = threadIdx.x; i < nv; i += kRedThreads) {
+      const uint4 w = __ldcs(p + i);
+      const T* e = reinterpret_cast<const T*>(&w);
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) {
+        const float x = to_f32(e[j]);
+        const uint64_t key = make_key(x, (uint32_t)(lo + i * VEC + j));
+        best = key > best ? key : best;
+        if (TYPICAL) soft_add(sf, x * zscale);
+      }
+    }
+  } else {
+    for (int i = lo + threadIdx.x; i < hi; i += kRedThreads) {
+      const float x = to_f32(xr[i]);
+      const uint64_t key = make_key(x, (uint32_t)i);
+      best = key > best ? key : best;
+      if (TYPICAL) soft_add(sf, x * zscale);
+    }
+  }
+  // block reduction
+  best = warp_max_u64(best);
+  if (TYPICAL) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      Soft other;
+      other.m = __shfl_xor_sync(0xffffffffu, sf.m, o);
+      other.Z = __shfl_xor_sync(0xffffffffu, sf.Z, o);
+      other.S = __shfl_xor_sync(0xffffffffu, sf.S, o);
+      sf = soft_merge(sf, other);
+    }
+  }
+  __shared__ uint64_t sk[kRedThreads / 32];
+  __shared__ Soft ss[kRedThreads / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    sk[warp] = best;
+    ss[warp] = sf;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < kRedThreads / 32; ++w) {
+      best = sk[w] > best ? sk[w] : best;
+      if (TYPICAL) sf = soft_merge(sf, ss[w]);
+    }
+    RowPart rp;
+    rp.key = best;
+    rp.m = sf.m;
+    rp.Z = sf.Z;
+    rp.S = sf.S;
+    rp.pad = 0.f;
+    parts[row * splits + sp] = rp;
+  }
+}
+
+template <typename T, bool TYPICAL>
+__global__ void __launch_bounds__(32)
+    accept_walk_kernel(const T* __restrict__ vlog, const RowPart* __restrict__ parts, int splits,
+                       const int32_t* __restrict__ tok, const int32_t* __restrict__ parent,
+                       const int32_t* __restrict__ depth, const uint32_t* __restrict__ anc, int N,
+                       int W, int K, int V, float zscale, float eps, float delta,
+                       int32_t* __restrict__ accept_len, int32_t* __restrict__ accept_nodes,
+                       int32_t* __restrict__ next_tok) {
+  __shared__ int32_t amax[MEDUSA_MAX_N];
+  __shared__ float mrow[MEDUSA_MAX_N], zrow[MEDUSA_MAX_N], thr[MEDUSA_MAX_N];
+  __shared__ uint32_t cond[MEDUSA_MAX_N / 32];
+  const int b = blockIdx.x;
+  const int lane = threadIdx.x;
+
+  for (int n = lane; n < N; n += 32) {
+    const RowPart* pr = parts + ((size_t)b * N + n) * splits;
+    uint64_t best = 0ull;
+    Soft sf{-INFINITY, 0.f, 0.f};
+    for (int s2 = 0; s2 < splits; ++s2) {
+      const RowPart rp = pr[s2];
+      best = rp.key > best ? rp.key : best;
+      if (TYPICAL) sf = soft_merge(sf, Soft{rp.m, rp.Z, rp.S});
+    }
+    amax[n] = (int32_t)key_index(best);
+    if (TYPICAL) {
+      mrow[n] = sf.m;
+      zrow[n] = sf.Z;
+      const float H = logf(sf.Z) - kLn2 * sf.S / sf.Z;
+      thr[n] = fminf(eps, delta * expf(-H));
+    }
+  }
+  __syncwarp();
+
+  // each node's own condition (root: true)
+  for (int n0 = 0; n0 < N; n0 += 32) {
+    const int n = n0 + lane;
+    bool c = (n == 0);
+    if (n > 0 && n < N) {
+      const int par = parent[n];
+      const int t = tok[(size_t)b * N + n];
+      if (TYPICAL) {
+        if (t >= 0 && t < V) {
+          const float x = to_f32(vlog[((size_t)b * N + par) * V + t]);
+          const float p = exp2f(x * zscale - mrow[par]) / zrow[par];
+          c = p > thr[par];
+        }
+      } else {
+        c = (amax[par] == t);
+      }
+    }
+    const uint32_t bits = __ballot_sync(0xffffffffu, c);
+    if (lane == 0) cond[n0 >> 5] = bits;
+  }
+  __syncwarp();
+
+  // accepted iff every node on the root path satisfies its condition;
+  // deepest accepted node wins, ties to the lowest index.
+  uint32_t key = 0u;
+  for (int n = lane; n < N; n += 32) {
+    bool ok = true;
+    for (int w = 0; w < W; ++w) ok = ok && ((anc[(size_t)n * W + w] & ~cond[w]) == 0u);
+    if (ok) {
+      const uint32_t k2 = ((uint32_t)depth[n] << 16) | (0xFFFFu - (uint32_t)n);
+      key = k2 > key ? k2 : key;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint32_t other = __shfl_xor_sync(0xffffffffu, key, o);
+    key = other > key ? other : key;
+  }
+  const int best = (int)(0xFFFFu - (key & 0xFFFFu));
+  const int D = (int)(key >> 16);
+  if (lane == 0) {
+    accept_len[b] = D;
+    next_tok[b] = amax[best];
+    int j = 0;
+    for (int w = 0; w < W; ++w) {
+      uint32_t bits = anc[(size_t)best * W + w];
+      while (bits) {
+        const int i = __ffs(bits) - 1;
+        bits &= bits - 1;
+        if (j <= K) accept_nodes[(size_t)b * (K + 1) + j] = w * 32 + i;
+        ++j;
+      }
+    }
+    for (; j <= K; ++j) accept_nodes[(size_t)b * (K + 1) + j] = -1;
+  }
+}
+
+struct AccPlan {
+  int splits, chunk;
+  size_t total;
+};
+
+AccPlan make_plan(int rows, int V) {
+  AccPlan P;
+  const int target = 4 * num_sms();
+  int splits = (target + rows - 1) / (rows > 0 ? rows : 1);
+  const int max_splits = (V + 2047) / 2048;  // keep >= ~2K elements per CTA
+  splits = splits < 1 ? 1 : (splits > max_splits ? max_splits : splits);
+  splits = splits < 1 ? 1 : splits;
+  int chunk = (V + splits - 1) / splits;
+  chunk = (chunk + 7) & ~7;  // 16-byte aligned chunk starts for bf16 rows
+  splits = (V + chunk - 1) / chunk;
+  P.splits = splits;
+  P.chunk = chunk;
+  WsCarver w;
+  w.take<RowPart>((size_t)rows * splits);
+  P.total = w.total();
+  return P;
+}
+
+}  // namespace
+
+size_t accept_workspace(const medusa_tree* t, int B, int V) {
+  return make_plan(B * t->N, V).total;
+}
+
+int accept_launch(const AcceptArgs& a, cudaStream_t st) {
+  const int N = a.tree->N;
+  const int rows = a.B * N;
+  if (rows == 0) return MEDUSA_OK;
+  const AccPlan P = make_plan(rows, a.V);
+  if (a.ws_bytes < P.total) return fail(MEDUSA_ERR_INVALID_ARG, "workspace too small for accept");
+  RowPart* parts = (RowPart*)a.ws;
+  const float zscale = a.typical ? kLog2e / a.temperature : 0.f;
+  dim3 g1(rows, P.splits);
+  const medusa_tree* t = a.tree;
+#define MEDUSA_ACC(T, TYP)                                                                    \
+  do {                                                                                        \
+    row_reduce_kernel<T, TYP><<<g1, kRedThreads, 0, st>>>((const T*)a.vlog, a.V, P.chunk,     \
+                                                          P.splits, zscale, parts);           \
+    accept_walk_kernel<T, TYP><<<a.B, 32, 0, st>>>(                                           \
+        (const T*)a.vlog, parts, P.splits, a.tok, t->d_parent, t->d_depth, t->d_anc, N, t->W, \
+        t->K, a.V, zscale, a.eps, a.delta, a.accept_len, a.accept_nodes, a.next_tok);         \
+  } while (0)
+  if (a.dtype == MEDUSA_F32) {
+    if (a.typical) MEDUSA_ACC(float, true);
+    else MEDUSA_ACC(float, false);
+  } else {
+    if (a.typical) MEDUSA_ACC(__nv_bfloat16, true);
+    else MEDUSA_ACC(__nv_bfloat16, false);
+  }
+#undef MEDUSA_ACC
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "accept kernels launch");
+}
+
+}  // namespace medusa

@@ -1,0 +1,122 @@
+// Internal declarations shared by the host API and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "../../include/medusa.h"
+
+struct medusa_tree {
+  int K = 0, s = 0, N = 0, W = 0;  // W = 32-bit words per ancestor-mask row
+  int device = -1;
+  std::vector<int32_t> parent, depth, rank_path, head_rank;
+  std::vector<uint32_t> anc;
+  // device copies (one allocation owned by the plan)
+  void* d_block = nullptr;
+  const int32_t* d_parent = nullptr;
+  const int32_t* d_depth = nullptr;
+  const int32_t* d_head_rank = nullptr;  // (D-1)*s + r_D, -1 for the root
+  const uint32_t* d_anc = nullptr;
+};
+
+namespace medusa {
+
+// Thread-local error message plumbing (defined in medusa_api.cu).
+int fail(int code, const std::string& msg);
+int cuda_fail(cudaError_t e, const char* what);
+int num_sms();
+
+// Carves 256-byte-aligned segments out of a caller workspace.
+struct WsCarver {
+  size_t off = 0;
+  template <typename T>
+  size_t take(size_t count) {
+    off = (off + 255) & ~(size_t)255;
+    size_t at = off;
+    off += count * sizeof(T);
+    return at;
+  }
+  size_t total() const { return (off + 255) & ~(size_t)255; }
+};
+
+// ---------------------------------------------------------------- heads
+struct HeadsArgs {
+  const void* h;
+  const void* W1;
+  const void* b1;
+  const void* W2;
+  int B, d, V, K, dtype;
+  float* logits;
+  int s;
+  int32_t* topk_idx;
+  float* topk_val;
+  void* ws;
+  size_t ws_bytes;
+};
+size_t heads_tc_workspace(int B, int d, int V, int K, int s);
+int heads_tc_launch(const HeadsArgs& a, cudaStream_t st);
+size_t heads_simt_workspace(int B, int d, int V, int K, int s);
+int heads_simt_launch(const HeadsArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------- top-s
+int topk_rows_launch(const void* x, int dtype, int R, int V, int s, int32_t* idx, float* val,
+                     cudaStream_t st);
+int topk_keys_launch(const uint64_t* keys, int R, int C, int s, int32_t* idx, float* val,
+                     cudaStream_t st);
+
+// ---------------------------------------------------------------- tree
+int build_tree_launch(const medusa_tree* t, const int32_t* root, const int32_t* topk,
+                      const int32_t* L, int B, int32_t* tok, int32_t* pos, cudaStream_t st);
+
+// ---------------------------------------------------------------- attention
+struct AttnArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const int32_t* L;
+  const medusa_tree* tree;
+  int B, Hq, Hkv, dh, Lcap;
+  float scale;
+  int dtype;
+  void* out;
+  void* ws;
+  size_t ws_bytes;
+};
+size_t attention_workspace(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lcap,
+                           int dtype);
+int attention_launch(const AttnArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------- acceptance
+struct AcceptArgs {
+  const void* vlog;
+  int dtype;
+  const int32_t* tok;
+  const medusa_tree* tree;
+  int B, V;
+  bool typical;
+  float temperature, eps, delta;
+  int32_t* accept_len;
+  int32_t* accept_nodes;
+  int32_t* next_tok;
+  void* ws;
+  size_t ws_bytes;
+};
+size_t accept_workspace(const medusa_tree* t, int B, int V);
+int accept_launch(const AcceptArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------- compaction
+int kv_compact_launch(void* k, void* v, const int32_t* L, const int32_t* alen,
+                      const int32_t* anodes, int B, int Hkv, int dh, int Lcap, int K,
+                      int dtype, int32_t* new_len, cudaStream_t st);
+
+// ---------------------------------------------------------------- TMA descriptors
+// Encodes a bf16 tensor map (dims innermost first) with 128-byte swizzling.
+int make_tmap_bf16(void* map /* CUtensorMap* */, const void* base, int rank,
+                   const uint64_t* dims, const uint64_t* strides_bytes,
+                   const uint32_t* box);
+
+}  // namespace medusa

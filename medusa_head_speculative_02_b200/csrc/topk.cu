@@ -1,0 +1,111 @@
+// Top-s selection.  Medusa paper digest ("論文解説: Medusa"), section
+// "ツリーアテンションによる並列検証": each head contributes its s most likely
+// tokens.  Order: value descending, ties to the lower index, encoded in one
+// 64-bit key per element so a single unsigned compare decides.
+//
+// One CTA per row: every thread keeps a sorted register list of its best s
+// keys while streaming its strided share of the row (16-byte vector loads
+// when the row is aligned), then s rounds of a block-wide max pop the winners.
+#include "common.cuh"
+#include "internal.h"
+
+namespace medusa {
+namespace {
+
+constexpr int kSmax = MEDUSA_MAX_S;
+constexpr int kThreads = 256;
+
+// s rounds: block max of every thread's best remaining key; the owner pops it.
+__device__ __forceinline__ void block_select(uint64_t (&k)[kSmax], int s, uint64_t* red, int32_t* idx_out,
+                             float* val_out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int j = 0; j < s; ++j) {
+    const uint64_t m = warp_max_u64(k[0]);
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    uint64_t best = red[0];
+#pragma unroll
+    for (int w = 1; w < kThreads / 32; ++w) best = red[w] > best ? red[w] : best;
+    if (best != 0ull && k[0] == best) topk_pop<kSmax>(k);
+    if (threadIdx.x == 0) {
+      idx_out[j] = best ? (int32_t)key_index(best) : -1;
+      if (val_out) val_out[j] = best ? key_value(best) : __int_as_float(0x7fc00000);
+    }
+    __syncthreads();
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) topk_rows_kernel(const T* __restrict__ x, int V, int s,
+                                                             int32_t* __restrict__ idx,
+                                                             float* __restrict__ val) {
+  __shared__ uint64_t red[kThreads / 32];
+  const size_t row = blockIdx.x;
+  const T* xr = x + row * (size_t)V;
+  uint64_t k[kSmax];
+#pragma unroll
+  for (int i = 0; i < kSmax; ++i) k[i] = 0ull;
+  uint64_t kth = 0ull;
+  constexpr int VEC = 16 / sizeof(T);
+  if ((V % VEC) == 0 && (((uintptr_t)xr) & 15u) == 0) {
+    const int nv = V / VEC;
+    for (int i = threadIdx.x; i < nv; i += kThreads) {
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(xr) + i);
+      const T* e = reinterpret_cast<const T*>(&w);
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) {
+        const uint64_t key = make_key(to_f32(e[j]), (uint32_t)(i * VEC + j));
+        if (key > kth) topk_insert<kSmax>(k, s, key, kth);
+      }
+    }
+  } else {
+    for (int i = threadIdx.x; i < V; i += kThreads) {
+      const uint64_t key = make_key(to_f32(xr[i]), (uint32_t)i);
+      if (key > kth) topk_insert<kSmax>(k, s, key, kth);
+    }
+  }
+  block_select(k, s, red, idx + row * s, val ? val + row * s : nullptr);
+}
+
+// Rows of pre-built candidate keys (0 = empty).
+__global__ void __launch_bounds__(kThreads) topk_keys_kernel(const uint64_t* __restrict__ keys,
+                                                             int C, int s,
+                                                             int32_t* __restrict__ idx,
+                                                             float* __restrict__ val) {
+  __shared__ uint64_t red[kThreads / 32];
+  const size_t row = blockIdx.x;
+  const uint64_t* kr = keys + row * (size_t)C;
+  uint64_t k[kSmax];
+#pragma unroll
+  for (int i = 0; i < kSmax; ++i) k[i] = 0ull;
+  uint64_t kth = 0ull;
+  for (int i = threadIdx.x; i < C; i += kThreads) {
+    const uint64_t key = __ldcg(kr + i);
+    if (key > kth) topk_insert<kSmax>(k, s, key, kth);
+  }
+  block_select(k, s, red, idx + row * s, val ? val + row * s : nullptr);
+}
+
+}  // namespace
+
+int topk_rows_launch(const void* x, int dtype, int R, int V, int s, int32_t* idx, float* val,
+                     cudaStream_t st) {
+  if (R == 0) return MEDUSA_OK;
+  if (dtype == MEDUSA_F32)
+    topk_rows_kernel<float><<<R, kThreads, 0, st>>>((const float*)x, V, s, idx, val);
+  else
+    topk_rows_kernel<__nv_bfloat16><<<R, kThreads, 0, st>>>((const __nv_bfloat16*)x, V, s, idx,
+                                                            val);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "topk_rows_kernel launch");
+}
+
+int topk_keys_launch(const uint64_t* keys, int R, int C, int s, int32_t* idx, float* val,
+                     cudaStream_t st) {
+  if (R == 0) return MEDUSA_OK;
+  topk_keys_kernel<<<R, kThreads, 0, st>>>(keys, C, s, idx, val);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "topk_keys_kernel launch");
+}
+
+}  // namespace medusa

@@ -1,0 +1,162 @@
+"""One Medusa verify step through the public API, with preallocated buffers.
+
+A step is: heads (+ fused top-s) -> tree expansion -> tree attention ->
+acceptance (greedy, typical or both) -> KV compaction, all on the current
+CUDA stream.  ``HostIO`` adds the per-step host<->device traffic of a real
+decoder (hidden state, tree queries, tree K/V, verify logits and token ids
+in; acceptance results out) for end-to-end timing.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import api
+from .synthetic import MedusaConfig, gen_inputs, plant_verify_logits
+
+# kernels this library launches per call (host memsets excluded)
+LAUNCHES = {"heads": 3, "build_tree": 1, "tree_attention": 2, "accept": 2, "kv_compact": 1}
+
+
+class VerifyStep:
+    def __init__(self, cfg: MedusaConfig, device="cuda", seed: int = 0):
+        self.cfg = cfg
+        self.dev = torch.device(device)
+        self.x = gen_inputs(cfg, self.dev, seed)
+        self.tree = api.Tree(cfg.K, cfg.s, cfg.N)
+        B, K, s, N = cfg.B, cfg.K, cfg.s, cfg.N
+        i32 = dict(dtype=torch.int32, device=self.dev)
+        self.topk_idx = torch.empty(B, K, s, **i32)
+        self.topk_val = torch.empty(B, K, s, dtype=torch.float32, device=self.dev)
+        self.tree_tok = torch.empty(B, N, **i32)
+        self.tree_pos = torch.empty(B, N, **i32)
+        self.attn_out = torch.empty_like(self.x["q"])
+        self.accept_len = torch.empty(B, **i32)
+        self.accept_nodes = torch.empty(B, K + 1, **i32)
+        self.next_tok = torch.empty(B, **i32)
+        self.accept_len2 = torch.empty(B, **i32)
+        self.accept_nodes2 = torch.empty(B, K + 1, **i32)
+        self.next_tok2 = torch.empty(B, **i32)
+        self.new_len = torch.empty(B, **i32)
+        self.ws_heads = torch.empty(api.heads_workspace_size(B, cfg.d, cfg.V, K, s, cfg.torch_dtype),
+                                    dtype=torch.uint8, device=self.dev)
+        self.ws_attn = torch.empty(max(256, api.attention_workspace_size(self.tree, B, cfg.Hq,
+                                                                         cfg.Hkv, cfg.dh, cfg.Lcap)),
+                                   dtype=torch.uint8, device=self.dev)
+        self.ws_acc = torch.empty(max(256, api.accept_workspace_size(self.tree, B, cfg.V)),
+                                  dtype=torch.uint8, device=self.dev)
+        self.scale = 1.0 / math.sqrt(cfg.dh)
+        # verify logits are planted along the tree this step's heads produce
+        self.heads()
+        self.build_tree()
+        torch.cuda.synchronize(self.dev)
+        parent = self.tree.info()[0]
+        self.vlogits = plant_verify_logits(cfg, parent, self.tree_tok.cpu(), self.dev, seed)
+
+    # individual calls --------------------------------------------------------
+    def heads(self):
+        x = self.x
+        api.medusa_heads_forward(x["h"], x["W1"], x["b1"], x["W2"], s=self.cfg.s,
+                                 want_logits=False,
+                                 out=(None, self.topk_idx, self.topk_val), ws=self.ws_heads)
+
+    def build_tree(self):
+        api.medusa_build_tree(self.tree, self.x["root_tok"], self.topk_idx, self.x["prefix_len"],
+                              out=(self.tree_tok, self.tree_pos))
+
+    def attention(self):
+        x = self.x
+        api.medusa_tree_attention(x["q"], x["k_cache"], x["v_cache"], x["prefix_len"], self.tree,
+                                  self.scale, out=self.attn_out, ws=self.ws_attn)
+
+    def accept(self):
+        cfg = self.cfg
+        if cfg.accept in ("greedy", "both"):
+            api.medusa_accept_greedy(self.vlogits, self.tree_tok, self.tree,
+                                     out=(self.accept_len, self.accept_nodes, self.next_tok),
+                                     ws=self.ws_acc)
+        if cfg.accept in ("typical", "both"):
+            out = (self.accept_len, self.accept_nodes, self.next_tok) if cfg.accept == "typical" \
+                else (self.accept_len2, self.accept_nodes2, self.next_tok2)
+            api.medusa_accept_typical(self.vlogits, self.tree_tok, self.tree, cfg.temperature,
+                                      cfg.eps, cfg.delta, out=out, ws=self.ws_acc)
+
+    def compact(self):
+        x = self.x
+        api.medusa_kv_compact(x["k_cache"], x["v_cache"], x["prefix_len"], self.accept_len,
+                              self.accept_nodes, self.cfg.K, new_len=self.new_len)
+
+    def run(self):
+        self.heads()
+        self.build_tree()
+        self.attention()
+        self.accept()
+        self.compact()
+
+    def launches_per_step(self) -> int:
+        n_acc = 2 if self.cfg.accept == "both" else 1
+        return (LAUNCHES["heads"] + LAUNCHES["build_tree"] + LAUNCHES["tree_attention"] +
+                n_acc * LAUNCHES["accept"] + LAUNCHES["kv_compact"])
+
+    # algorithmic bytes --------------------------------------------------------
+    def heads_bytes(self) -> int:
+        c = self.cfg
+        e = 4 if c.dtype == "f32" else 2
+        return e * (c.K * c.d * c.d + c.K * c.d + c.K * c.V * c.d + c.B * c.d) + 8 * c.B * c.K * c.s
+
+    def attention_bytes(self) -> int:
+        """K/V actually read (prefix + tree slots) + Q + O."""
+        c = self.cfg
+        e = 4 if c.dtype == "f32" else 2
+        Lsum = int(self.x["prefix_len"].sum().item())
+        kv = 2 * (Lsum + c.B * c.N) * c.Hkv * c.dh * e
+        return kv + 2 * c.B * c.N * c.Hq * c.dh * e
+
+
+class HostIO:
+    """Pinned host copies of one step's per-step inputs and outputs."""
+
+    def __init__(self, st: VerifyStep):
+        self.st = st
+        c = st.cfg
+        x = st.x
+        pin = dict(pin_memory=True)
+        self.h = x["h"].cpu().pin_memory()
+        self.q = x["q"].cpu().pin_memory()
+        self.vlog = st.vlogits.cpu().pin_memory()
+        self.root = x["root_tok"].cpu().pin_memory()
+        self.plen = x["prefix_len"].cpu().pin_memory()
+        self.L = [int(v) for v in self.plen.tolist()]
+        self.tree_k = torch.stack([x["k_cache"][b, self.L[b]:self.L[b] + c.N] for b in range(c.B)]).cpu().pin_memory()
+        self.tree_v = torch.stack([x["v_cache"][b, self.L[b]:self.L[b] + c.N] for b in range(c.B)]).cpu().pin_memory()
+        self.o_alen = torch.empty(c.B, dtype=torch.int32, **pin)
+        self.o_nodes = torch.empty(c.B, c.K + 1, dtype=torch.int32, **pin)
+        self.o_next = torch.empty(c.B, dtype=torch.int32, **pin)
+        self.o_len = torch.empty(c.B, dtype=torch.int32, **pin)
+        self.o_topk = torch.empty(c.B, c.K, c.s, dtype=torch.int32, **pin)
+
+    def h2d_bytes(self) -> int:
+        ts = [self.h, self.q, self.vlog, self.root, self.plen, self.tree_k, self.tree_v]
+        return sum(t.numel() * t.element_size() for t in ts)
+
+    def d2h_bytes(self) -> int:
+        ts = [self.o_alen, self.o_nodes, self.o_next, self.o_len, self.o_topk]
+        return sum(t.numel() * t.element_size() for t in ts)
+
+    def step(self):
+        st, x, c = self.st, self.st.x, self.st.cfg
+        x["h"].copy_(self.h, non_blocking=True)
+        x["q"].copy_(self.q, non_blocking=True)
+        st.vlogits.copy_(self.vlog, non_blocking=True)
+        x["root_tok"].copy_(self.root, non_blocking=True)
+        x["prefix_len"].copy_(self.plen, non_blocking=True)
+        for b in range(c.B):
+            x["k_cache"][b, self.L[b]:self.L[b] + c.N].copy_(self.tree_k[b], non_blocking=True)
+            x["v_cache"][b, self.L[b]:self.L[b] + c.N].copy_(self.tree_v[b], non_blocking=True)
+        st.run()
+        self.o_alen.copy_(st.accept_len, non_blocking=True)
+        self.o_nodes.copy_(st.accept_nodes, non_blocking=True)
+        self.o_next.copy_(st.next_tok, non_blocking=True)
+        self.o_len.copy_(st.new_len, non_blocking=True)
+        self.o_topk.copy_(st.topk_idx, non_blocking=True)

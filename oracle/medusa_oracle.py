@@ -45,7 +45,7 @@ __all__ = [
     "f64", "tree_score", "tree_plan", "silu", "heads_forward", "topk_row",
     "topk", "build_tree", "tree_attention", "row_argmax", "accept_greedy",
     "typical_row_stats", "typical_threshold", "accept_typical", "kv_compact",
-    "ancestors_or_self",
+    "ancestors_or_self", "heads_hidden", "heads_logits",
 ]
 
 
@@ -160,12 +160,24 @@ def heads_forward(h, W1, b1, W2, heads=None, vocab=None) -> np.ndarray:
     vocab = np.arange(V) if vocab is None else np.asarray(vocab)
     out = np.zeros((hh.shape[0], len(heads), len(vocab)))
     for j, k in enumerate(heads):
-        a = hh @ f64(W1[k]).T
-        if b1 is not None:
-            a = a + f64(b1[k])[None, :]
-        u = silu(a) + hh
-        out[:, j, :] = u @ _rows(W2[k], vocab).T
+        out[:, j, :] = heads_logits(heads_hidden(hh, W1, b1, k), W2, k, vocab)
     return out
+
+
+def heads_hidden(h, W1, b1, k: int, rows=None) -> np.ndarray:
+    """u = SiLU(W1_k h + b1_k) + h for head k ([B][d], or [B][len(rows)])."""
+    hh = f64(h)
+    rows = np.arange(W1.shape[1]) if rows is None else np.asarray(rows)
+    a = hh @ _rows(W1[k], rows).T
+    if b1 is not None:
+        a = a + f64(b1[k])[rows][None, :]
+    return silu(a) + hh[:, rows]
+
+
+def heads_logits(u, W2, k: int, vocab=None) -> np.ndarray:
+    """logits = W2_k u for head k ([B][V], or [B][len(vocab)])."""
+    vocab = np.arange(W2.shape[1]) if vocab is None else np.asarray(vocab)
+    return f64(u) @ _rows(W2[k], vocab).T
 
 
 # ---------------------------------------------------------------------------
