@@ -139,7 +139,7 @@ def _attn_case(B, N_K_s, Hq, Hkv, dh, Ls, dtype, seed):
     (2, (5, 3, 100), 2, 2, 64, [33, 0], torch.float32),
 ])
 def test_tree_attention_small(B, tree, Hq, Hkv, dh, Ls, dtype):
-    K, s, N, q, kc, vc, L = _attn_case(B, tree, Hq, Hkv, dh, Ls, dtype, seed=B * 100 + N)
+    K, s, N, q, kc, vc, L = _attn_case(B, tree, Hq, Hkv, dh, Ls, dtype, seed=B * 100 + tree[2])
     t = api.Tree(K, s, N)
     plan = O.tree_plan(K, s, N)
     scale = 1.0 / math.sqrt(dh)
