@@ -214,6 +214,31 @@ int medusa_accept_typical(const void* vlogits, int dtype,
                           int32_t* accept_nodes, int32_t* next_tok, void* ws,
                           size_t ws_bytes, void* stream);
 
+/*
+ * medusa_accept_greedy without a workspace argument, for callers that cannot
+ * allocate device memory: code that runs where cudaMalloc and allocating
+ * libraries are off limits (for example a serving loop whose device memory
+ * was partitioned up front, or a host language binding with no device
+ * allocator of its own).  The paper has no counterpart; this is a library
+ * convenience.  Same inputs, outputs and results as medusa_accept_greedy.
+ * Its scratch is a fixed array inside the library of
+ * MEDUSA_NOALLOC_ACCEPT_PARTS row-chunk records (24 bytes each, 1.5 MiB),
+ * which every GPU that loads the library holds until the process exits.
+ * Limit: B * N <= MEDUSA_NOALLOC_ACCEPT_PARTS, else MEDUSA_ERR_INVALID_ARG
+ * and nothing is launched.  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress, host side, once per device); make
+ * that first call before any stream capture.  All calls share the array:
+ * calls that may overlap on the GPU (different streams without ordering)
+ * race and must be serialized by the caller.  No memory is allocated or
+ * freed by this call.
+ */
+#define MEDUSA_NOALLOC_ACCEPT_PARTS 65536
+int medusa_accept_greedy_noalloc(const void* vlogits, int dtype,
+                                 const int32_t* tree_tok,
+                                 const medusa_tree_t* tree, int B, int V,
+                                 int32_t* accept_len, int32_t* accept_nodes,
+                                 int32_t* next_tok, void* stream);
+
 /* ------------------------------------------------------------------------
  * KV compaction of the accepted path (the accepted tokens' K/V become the
  * contiguous continuation of the sequence):

@@ -17,6 +17,8 @@
 // accept a node iff its whole root path satisfies the condition (ancestor
 // bitmask test), take the deepest accepted node (ties: lowest index) and
 // emit its path and the argmax of its row.
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -285,6 +287,79 @@ int accept_launch(const AcceptArgs& a, cudaStream_t st) {
 #undef MEDUSA_ACC
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "accept kernels launch");
+}
+
+// ---------------------------------------------------------------------------
+// Greedy acceptance whose scratch is owned by the library, for callers that
+// cannot allocate device memory.  The per-row-chunk results of the verify
+// row reduction go to this fixed array instead of a caller workspace:
+// MEDUSA_NOALLOC_ACCEPT_PARTS entries x 24 bytes (1.5 MiB), held by every
+// GPU that loads the library until the process exits.  Every call writes
+// each entry it reads before reading it, so nothing has to start at zero;
+// calls that overlap on the GPU share the array and race.
+static __device__ __align__(256) RowPart g_accept_scratch[MEDUSA_NOALLOC_ACCEPT_PARTS];
+
+namespace {
+std::mutex g_scratch_mu;
+RowPart* g_scratch_addr[64] = {nullptr};
+
+// Device address of g_accept_scratch on the current device, looked up once
+// per device (with that device current) and cached.
+int scratch_address(RowPart** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(MEDUSA_ERR_UNSUPPORTED, "device ordinal >= 64");
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_accept_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_accept_scratch)");
+    g_scratch_addr[dev] = (RowPart*)p;
+  }
+  *out = g_scratch_addr[dev];
+  return MEDUSA_OK;
+}
+}  // namespace
+
+int accept_greedy_noalloc_launch(const void* vlog, int dtype, const int32_t* tok,
+                                 const medusa_tree* t, int B, int V, int32_t* accept_len,
+                                 int32_t* accept_nodes, int32_t* next_tok, cudaStream_t st) {
+  const int N = t->N;
+  const long long rows = (long long)B * N;
+  if (rows == 0) return MEDUSA_OK;
+  if (rows > MEDUSA_NOALLOC_ACCEPT_PARTS)
+    return fail(MEDUSA_ERR_INVALID_ARG,
+                "medusa_accept_greedy_noalloc: B*N exceeds its static scratch "
+                "(MEDUSA_NOALLOC_ACCEPT_PARTS rows)");
+  AccPlan P = make_plan((int)rows, V);
+  if (rows * P.splits > MEDUSA_NOALLOC_ACCEPT_PARTS) {
+    // fewer, longer chunks per row so every (row, chunk) result fits
+    const int splits = (int)(MEDUSA_NOALLOC_ACCEPT_PARTS / rows);
+    int chunk = (V + splits - 1) / splits;
+    chunk = (chunk + 7) & ~7;
+    P.chunk = chunk;
+    P.splits = (V + chunk - 1) / chunk;
+  }
+  RowPart* parts = nullptr;
+  int rc = scratch_address(&parts);
+  if (rc) return rc;
+  dim3 g1((unsigned)rows, P.splits);
+#define MEDUSA_ACC_STATIC(T)                                                                    \
+  do {                                                                                          \
+    row_reduce_kernel<T, false><<<g1, kRedThreads, 0, st>>>((const T*)vlog, V, P.chunk,         \
+                                                            P.splits, 0.f, parts);              \
+    accept_walk_kernel<T, false><<<B, 32, 0, st>>>(                                             \
+        (const T*)vlog, parts, P.splits, tok, t->d_parent, t->d_depth, t->d_anc, N, t->W, t->K, \
+        V, 0.f, 0.f, 0.f, accept_len, accept_nodes, next_tok);                                  \
+  } while (0)
+  if (dtype == MEDUSA_F32)
+    MEDUSA_ACC_STATIC(float);
+  else
+    MEDUSA_ACC_STATIC(__nv_bfloat16);
+#undef MEDUSA_ACC_STATIC
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "accept kernels launch (static scratch)");
 }
 
 }  // namespace medusa

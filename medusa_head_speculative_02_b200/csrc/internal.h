@@ -107,6 +107,9 @@ struct AcceptArgs {
 };
 size_t accept_workspace(const medusa_tree* t, int B, int V);
 int accept_launch(const AcceptArgs& a, cudaStream_t st);
+int accept_greedy_noalloc_launch(const void* vlog, int dtype, const int32_t* tok,
+                                 const medusa_tree* t, int B, int V, int32_t* accept_len,
+                                 int32_t* accept_nodes, int32_t* next_tok, cudaStream_t st);
 
 // ---------------------------------------------------------------- compaction
 int kv_compact_launch(void* k, void* v, const int32_t* L, const int32_t* alen,

@@ -445,6 +445,20 @@ int medusa_accept_typical(const void* vlogits, int dtype, const int32_t* tree_to
                        accept_len, accept_nodes, next_tok, ws, ws_bytes, stream);
 }
 
+int medusa_accept_greedy_noalloc(const void* vlogits, int dtype, const int32_t* tree_tok,
+                                 const medusa_tree_t* tree, int B, int V, int32_t* accept_len,
+                                 int32_t* accept_nodes, int32_t* next_tok, void* stream) {
+  int rc = check_tree(tree);
+  if (rc) return rc;
+  if (!dtype_ok(dtype)) return fail(MEDUSA_ERR_INVALID_ARG, "bad dtype");
+  if (B < 0 || V < 1) return fail(MEDUSA_ERR_INVALID_ARG, "bad shape");
+  if (B == 0) return MEDUSA_OK;
+  if (!vlogits || !tree_tok || !accept_len || !accept_nodes || !next_tok)
+    return fail(MEDUSA_ERR_INVALID_ARG, "NULL pointer");
+  return accept_greedy_noalloc_launch(vlogits, dtype, tree_tok, tree, B, V, accept_len,
+                                      accept_nodes, next_tok, (cudaStream_t)stream);
+}
+
 int medusa_kv_compact(void* k_cache, void* v_cache, const int32_t* prefix_len,
                       const int32_t* accept_len, const int32_t* accept_nodes, int B, int Hkv,
                       int dh, int Lcap, int K, int dtype, int32_t* new_len, void* stream) {
