@@ -228,13 +228,52 @@ __global__ void tree_attn_combine_kernel(const float* __restrict__ po,
 
 }  // namespace
 
+namespace {
+// Partial-output layout of the tensor-core path (only used with > 1 chunk).
+struct TcPlan {
+  int P;
+  size_t off_o, off_ml, total;
+};
+TcPlan make_tc_plan(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lcap) {
+  TcPlan P;
+  P.P = attention_tc_chunks(B, Hq, Hkv, t->N, Lcap);
+  WsCarver w;
+  const size_t rows = P.P > 1 ? (size_t)B * Hkv * P.P * t->N * (Hq / Hkv) : 0;
+  P.off_o = w.take<float>(rows * dh);
+  P.off_ml = w.take<float2>(rows);
+  P.total = w.total();
+  return P;
+}
+}  // namespace
+
 size_t attention_workspace(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lcap,
-                           int /*dtype*/) {
-  return make_plan(t, B, Hq, Hkv, dh, Lcap).total;
+                           int dtype) {
+  const size_t simt = make_plan(t, B, Hq, Hkv, dh, Lcap).total;
+  const size_t tc = attention_tc_eligible(MEDUSA_BF16, dh, Hq, Hkv)
+                        ? make_tc_plan(t, B, Hq, Hkv, dh, Lcap).total
+                        : 0;
+  if (dtype < 0) return simt > tc ? simt : tc;  // size query without a dtype
+  return attention_tc_eligible(dtype, dh, Hq, Hkv) ? tc : simt;
 }
 
 int attention_launch(const AttnArgs& a, cudaStream_t st) {
   const medusa_tree* t = a.tree;
+  if (attention_tc_eligible(a.dtype, a.dh, a.Hq, a.Hkv)) {
+    const TcPlan P = make_tc_plan(t, a.B, a.Hq, a.Hkv, a.dh, a.Lcap);
+    if (a.ws_bytes < P.total)
+      return fail(MEDUSA_ERR_INVALID_ARG, "workspace too small for attention");
+    if (a.B == 0) return MEDUSA_OK;
+    float* po = (float*)((uint8_t*)a.ws + P.off_o);
+    float2* pml = (float2*)((uint8_t*)a.ws + P.off_ml);
+    int rc = attention_tc_run(a, P.P, po, pml, st);
+    if (rc || P.P == 1) return rc;
+    const int R = t->N * (a.Hq / a.Hkv);
+    const int rows = a.B * t->N * a.Hq;
+    tree_attn_combine_kernel<__nv_bfloat16, 128><<<(rows + 7) / 8, 256, 0, st>>>(
+        po, pml, a.L, a.B, t->N, a.Hq, a.Hkv, a.Lcap, P.P, R, (__nv_bfloat16*)a.out);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "tree attention combine launch");
+  }
   const AttnPlan P = make_plan(t, a.B, a.Hq, a.Hkv, a.dh, a.Lcap);
   if (a.ws_bytes < P.total) return fail(MEDUSA_ERR_INVALID_ARG, "workspace too small for attention");
   if (a.B == 0) return MEDUSA_OK;

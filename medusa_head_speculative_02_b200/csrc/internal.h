@@ -89,6 +89,10 @@ struct AttnArgs {
 size_t attention_workspace(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lcap,
                            int dtype);
 int attention_launch(const AttnArgs& a, cudaStream_t st);
+// tcgen05 path (bf16, dh = 128, GQA group dividing 128)
+bool attention_tc_eligible(int dtype, int dh, int Hq, int Hkv);
+int attention_tc_chunks(int B, int Hq, int Hkv, int N, int Lcap);
+int attention_tc_run(const AttnArgs& a, int P, float* po, float2* pml, cudaStream_t st);
 
 // ---------------------------------------------------------------- acceptance
 struct AcceptArgs {

@@ -379,7 +379,7 @@ int medusa_build_tree(const medusa_tree_t* tree, const int32_t* root_tok,
 size_t medusa_tree_attention_workspace_size(const medusa_tree_t* tree, int B, int Hq, int Hkv,
                                             int dh, int Lcap) {
   if (!tree || B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || Lcap < 0) return 0;
-  return attention_workspace(tree, B, Hq, Hkv, dh, Lcap, MEDUSA_BF16);
+  return attention_workspace(tree, B, Hq, Hkv, dh, Lcap, -1);
 }
 
 int medusa_tree_attention(const void* q, const void* k_cache, const void* v_cache,

@@ -137,6 +137,9 @@ def _attn_case(B, N_K_s, Hq, Hkv, dh, Ls, dtype, seed):
     (2, (5, 10, 64), 4, 1, 128, [300, 1000], torch.bfloat16),
     (1, (1, 1, 1), 2, 2, 128, [257], torch.bfloat16),
     (2, (5, 3, 100), 2, 2, 64, [33, 0], torch.float32),
+    (2, (5, 8, 128), 8, 2, 128, [1000, 777], torch.bfloat16),    # 4 row tiles, split keys
+    (1, (5, 3, 256), 2, 2, 128, [513], torch.bfloat16),          # two tree tiles
+    (2, (4, 4, 40), 16, 1, 128, [2100, 64], torch.bfloat16),     # GQA group 16
 ])
 def test_tree_attention_small(B, tree, Hq, Hkv, dh, Ls, dtype):
     K, s, N, q, kc, vc, L = _attn_case(B, tree, Hq, Hkv, dh, Ls, dtype, seed=B * 100 + tree[2])
