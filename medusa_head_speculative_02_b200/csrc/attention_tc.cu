@@ -37,7 +37,7 @@ constexpr int BN = 128;  // keys per tile
 constexpr int DH = 128;
 constexpr uint32_t HALF = 128 * 64 * 2;  // one 64-column half of a 128-row bf16 tile
 constexpr uint32_t TILE = 2 * HALF;      // 32 KB
-constexpr size_t SMEM = 1024 + 6 * (size_t)TILE + 256;
+constexpr size_t SMEM = 1024 + 7 * (size_t)TILE + 256;  // Q | K[2] | V[2] | P[2] | barriers
 constexpr float kRescale = 8.0f;  // log2 of the growth that forces a rescale
 
 struct TcAttnParams {
@@ -102,8 +102,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = sm;
   uint8_t* sK = sm + TILE;
   uint8_t* sV = sm + 3 * TILE;
-  uint8_t* sP = sm + 5 * TILE;
-  uint64_t* bars = (uint64_t*)(sm + 6 * TILE);
+  uint8_t* sP = sm + 5 * TILE;  // [2]
+  uint64_t* bars = (uint64_t*)(sm + 7 * TILE);
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;   // [2]
   uint64_t* k_empty = bars + 3;  // [2]
@@ -111,10 +111,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_empty = bars + 7;  // [2]
   uint64_t* s_full = bars + 9;   // [2]
   uint64_t* s_free = bars + 11;  // [2]
-  uint64_t* p_full = bars + 13;
-  uint64_t* o_done = bars + 14;
-  uint64_t* mma_done = bars + 15;
-  uint32_t* tmem_slot = (uint32_t*)(bars + 16);
+  uint64_t* p_full = bars + 13;  // [2] softmax wrote P buffer i
+  uint64_t* p_free = bars + 15;  // [2] the P.V reading P buffer i completed
+  uint64_t* o_done = bars + 17;  // every P.V completed (O stable for rescaling)
+  uint64_t* o_final = bars + 18; // the last P.V completed
+  uint64_t* mma_done = bars + 19;
+  uint32_t* tmem_slot = (uint32_t*)(bars + 20);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
   const int mt = blockIdx.x, chunk = blockIdx.y, bk = blockIdx.z;
@@ -143,8 +145,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 128);
     }
-    mbar_init(p_full, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&p_full[i], 4);
+      mbar_init(&p_free[i], 1);
+    }
     mbar_init(o_done, 1);
+    mbar_init(o_final, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -225,19 +231,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j >= 1) {
           const int jj = j - 1;
           const int st = jj & 1;
-          if (!mbar_wait(p_full, (uint32_t)(jj & 1), abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&p_full[jj & 1], (uint32_t)((jj >> 1) & 1), abort_flag)) { ok = false; break; }
           if (!mbar_wait(&v_full[st], (jj >> 1) & 1u, abort_flag)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
             const uint32_t aoff = (uint32_t)(kk >> 2) * HALF + (uint32_t)(kk & 3) * 32u;
-            umma_bf16(tO, umma_desc_sw128_kmajor(smem_u32(sP) + aoff),
+            umma_bf16(tO, umma_desc_sw128_kmajor(smem_u32(sP + (jj & 1) * TILE) + aoff),
                       umma_desc_sw128(smem_u32(sV + st * TILE) + (uint32_t)kk * 2048u, HALF,
                                       1024u),
                       idesc_o, (jj > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&v_empty[st]);
+          umma_commit(&p_free[jj & 1]);
           umma_commit(o_done);
+          if (jj == T - 1) umma_commit(o_final);
         }
       }
       umma_commit(mma_done);
@@ -263,62 +271,76 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       float s[BN];
 #pragma unroll
-      for (int c0 = 0; c0 < BN; c0 += 16) {
-        float t[16];
-        tmem_ld16(tmem + lane_base + (uint32_t)st * BN + c0, t);
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        float t[32];
+        tmem_ld32(tmem + lane_base + (uint32_t)st * BN + c0, t);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) s[c0 + e] = t[e];
+        for (int e = 0; e < 32; ++e) s[c0 + e] = t[e];
       }
       tc_fence_before();
       mbar_arrive(&s_free[st]);
 
-      // scale to base 2 and mask
-      float tmax = -INFINITY;
+      // mask (masked scores become -inf; full prefix tiles need none)
       if (j < rg.n_pre) {
         const int lim = rg.k_hi - (rg.k_lo + j * BN);
+        if (lim < BN) {
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          const float x = (c < lim) ? s[c] * p.qscale : -INFINITY;
-          s[c] = x;
-          tmax = fmaxf(tmax, x);
+          for (int c = 0; c < BN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
         }
       } else {
         const int tt = j - rg.n_pre;  // tree tile: nodes tt*128 .. tt*128+127
         uint32_t wsel[BN / 32];
 #pragma unroll
         for (int w = 0; w < BN / 32; ++w) wsel[w] = tt == 0 ? am[w] : am[BN / 32 + w];
+        const int nvalid = p.N - tt * BN;  // columns >= nvalid are past the last node
 #pragma unroll
         for (int c = 0; c < BN; ++c) {
-          const int jn = tt * BN + c;
-          const bool vis = jn < p.N && ((wsel[c >> 5] >> (c & 31)) & 1u);
-          const float x = vis ? s[c] * p.qscale : -INFINITY;
-          s[c] = x;
-          tmax = fmaxf(tmax, x);
+          const bool vis = c < nvalid && ((wsel[c >> 5] >> (c & 31)) & 1u);
+          s[c] = vis ? s[c] : -INFINITY;
         }
       }
+      // raw row max (8 independent chains), then base 2: scale > 0
+      float mx[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx[e] = s[e];
+#pragma unroll
+      for (int c = 8; c < BN; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
+      const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * p.qscale;
       float corr = 1.f;
       bool rescale = false;
       if (tmax > m_used + kRescale) {
-        corr = exp2f(m_used - tmax);  // 0 when m_used is -inf
+        corr = ex2_approx(m_used - tmax);  // 0 when m_used is -inf
         m_used = tmax;
         l *= corr;
         rescale = true;
       }
-      float rowsum = 0.f;
+      // p = 2^(scale*s - m); a row with no visible key yet has m = -inf and
+      // only -inf scores, for which 2^(-inf) = 0 with any finite offset
+      const float moff = (m_used == -INFINITY) ? 0.f : m_used;
+      float sum8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sum8[e] = 0.f;
 #pragma unroll
       for (int c = 0; c < BN; ++c) {
-        const float e = (s[c] == -INFINITY) ? 0.f : exp2f(s[c] - m_used);
+        const float e = ex2_approx(fmaf(s[c], p.qscale, -moff));
         s[c] = e;
-        rowsum += e;
+        sum8[c & 7] += e;
       }
-      l += rowsum;
+      l += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
 
-      // PV(j-1) must be done before P is overwritten or O rescaled
-      if (j >= 1) {
+      // P buffer j&1 is free once PV(j-2) has read it
+      if (j >= 2) {
+        ok = mbar_wait(&p_free[st], (uint32_t)(((j >> 1) & 1) ^ 1), abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      }
+      // rescaling O needs PV(j-1) complete (PV(j-2) is, so o_done is at most
+      // one completion away from the awaited one)
+      if (j >= 1 && __any_sync(0xffffffffu, rescale)) {
         ok = mbar_wait(o_done, (uint32_t)((j - 1) & 1), abort_flag);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale)) {
+        {
           const uint32_t tO = tmem + lane_base + 256;
 #pragma unroll
           for (int c0 = 0; c0 < DH; c0 += 16) {
@@ -339,28 +361,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             v2[e] = __floats2bfloat162_rn(s[h * 64 + c8 * 8 + 2 * e], s[h * 64 + c8 * 8 + 2 * e + 1]);
-          uint8_t* dst = sP + h * HALF + r * 128 + ((c8 ^ (r & 7)) << 4);
+          uint8_t* dst = sP + st * TILE + h * HALF + r * 128 + ((c8 ^ (r & 7)) << 4);
           *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(v2);
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[st]);
     }
     if (ok) {
-      ok = mbar_wait(o_done, (uint32_t)((T - 1) & 1), abort_flag);
+      ok = mbar_wait(o_final, 0u, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
       tc_fence_after();
       float o[DH];
 #pragma unroll
-      for (int c0 = 0; c0 < DH; c0 += 16) {
-        float t[16];
-        tmem_ld16(tmem + lane_base + 256 + c0, t);
+      for (int c0 = 0; c0 < DH; c0 += 32) {
+        float t[32];
+        tmem_ld32(tmem + lane_base + 256 + c0, t);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) o[c0 + e] = t[e];
+        for (int e = 0; e < 32; ++e) o[c0 + e] = t[e];
       }
       if (row_ok) write_row(p, b, kvh, chunk, grow, m_used, l, o, true);
     }

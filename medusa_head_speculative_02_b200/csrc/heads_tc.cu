@@ -18,15 +18,18 @@
 //   warp 1     single-thread tcgen05.mma issuer, fp32 accumulators in TMEM,
 //              double-buffered so the epilogue of one tile overlaps the next
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator (thread = output row)
-// Work units are (head, 128-row tile, K-split).  With more than one split
-// the partial sums go to scratch and the CTA that completes a tile last
-// (atomic ticket) sums them in split order (deterministic) and runs the
-// epilogue.  Stage 1's epilogue fuses bias + SiLU + residual and writes u as
-// a bf16 hi/lo pair (u = hi + lo, columns 2b and 2b+1 of stage 2's B
-// operand), so stage 2 sees u with ~16 significant bits.  Stage 2's epilogue
-// fuses the optional fp32 logits store and a warp-level top-s over each
-// 32-row slice (64-bit keys: value desc, index asc); a small merge kernel
-// selects the final top-s per (b, head).
+// Work units are (head, 128-row tile, K-split), the split count chosen so
+// the units fill the SMs' waves.  Stage 1 (few tiles: d rows per head)
+// writes each split's partial sums with plain stores; heads_silu_kernel then
+// sums the splits in order (deterministic) and applies bias + SiLU +
+// residual, writing u as a bf16 hi/lo pair (u = hi + lo, columns 2b and
+// 2b+1 of stage 2's B operand) so stage 2 sees u with ~16 significant bits.
+// Stage 2 (many tiles) normally runs unsplit; when it is split, the CTA that
+// completes a tile last (atomic ticket) sums the partials in split order.
+// Its epilogue fuses the optional fp32 logits store and the top-s: a warp
+// max over 64-bit keys (value desc, index asc) per 32-row slice, then the 4
+// slices merged per 128-row tile in shared memory; a small kernel selects
+// the final top-s of every (b, head) from the per-tile lists.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -46,7 +49,8 @@ struct TcCfg {
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = (200 * 1024) / STAGE_BYTES;
   static constexpr uint32_t TMEM_COLS = (2 * NC < 32) ? 32 : 2 * NC;
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 512;
+  static constexpr uint32_t CBUF_BYTES = (NC / 2) * 4 * MEDUSA_MAX_S * 8;  // per-tile top-s lists
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 512 + CBUF_BYTES;
 };
 
 struct TcParams {
@@ -97,6 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   volatile int* last_flag = (volatile int*)(tmem_slot + 2);
+  uint64_t* cbuf = (uint64_t*)((uint8_t*)full + 512);  // [B][4 warps][s] candidate keys
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -227,6 +232,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
 
+      const int m = mt * BM + r;  // output row within the head
+      if (p.stage == 1) {
+        // partial sums of this K-split, [split][head][b][d]; bias, SiLU and
+        // the residual are applied by heads_silu_kernel once all splits land
+        if (m < p.rows) {
+          float* dst = p.part + (((size_t)sp * p.K + kh) * p.B) * p.d + m;
+#pragma unroll
+          for (int b = 0; b < NC; ++b)
+            if (b < p.B) dst[(size_t)b * p.d] = v[b];
+        }
+        continue;
+      }
+
       if (p.splits > 1) {
         float* mine = p.part + ((size_t)tile * p.splits + sp) * p.ncp * BM;
 #pragma unroll
@@ -253,24 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
 
-      const int m = mt * BM + r;  // output row within the head
-      if (p.stage == 1) {
-        if (m < p.rows) {
-          const float bias = p.b1 ? __bfloat162float(p.b1[(size_t)kh * p.d + m]) : 0.f;
-#pragma unroll
-          for (int b = 0; b < NC; ++b) {
-            if (b < p.B) {
-              const float a = v[b] + bias;
-              const float uu = a / (1.f + expf(-a)) + __bfloat162float(p.h[(size_t)b * p.d + m]);
-              const __nv_bfloat16 hi = __float2bfloat16_rn(uu);
-              const __nv_bfloat16 lo = __float2bfloat16_rn(uu - __bfloat162float(hi));
-              __nv_bfloat16* urow = p.u + ((size_t)kh * 2 * p.B + 2 * b) * p.d + m;
-              urow[0] = hi;
-              urow[p.d] = lo;
-            }
-          }
-        }
-      } else {
+      {
         const bool valid = m < p.rows;
 #pragma unroll
         for (int b = 0; b < NC / 2; ++b) {
@@ -278,6 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float lg = v[2 * b] + v[2 * b + 1];
             if (p.logits && valid) p.logits[((size_t)b * p.K + kh) * p.rows + m] = lg;
             if (p.cand) {
+              // this warp's 32 rows: s rounds of a warp max over 64-bit keys
               uint64_t key = valid ? make_key(lg, (uint32_t)m) : 0ull;
               uint64_t keep = 0ull;
               for (int j = 0; j < p.s; ++j) {
@@ -285,10 +287,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (key == mx) key = 0ull;
                 if (lane == j) keep = mx;
               }
-              if (lane < p.s)
-                p.cand[(((size_t)b * p.K + kh) * ((size_t)p.mtiles * 4) + (size_t)mt * 4 + q) *
-                           p.s + lane] = keep;
+              if (lane < p.s) cbuf[(b * 4 + q) * p.s + lane] = keep;
             }
+          }
+        }
+        if (p.cand) {
+          // merge the 4 warps' lists: the tile's top-s per column b
+          named_bar_sync(1, 128);
+          for (int b = warp - 2; b < p.B; b += 4) {
+            uint64_t k0 = lane < 2 * p.s ? cbuf[b * 4 * p.s + lane] : 0ull;
+            uint64_t k1 = lane < 2 * p.s ? cbuf[b * 4 * p.s + 2 * p.s + lane] : 0ull;
+            uint64_t keep = 0ull;
+            for (int j = 0; j < p.s; ++j) {
+              const uint64_t mx = warp_max_u64(k0 > k1 ? k0 : k1);
+              if (k0 == mx) k0 = 0ull;
+              if (k1 == mx) k1 = 0ull;
+              if (lane == j) keep = mx;
+            }
+            if (lane < p.s)
+              p.cand[(((size_t)b * p.K + kh) * (size_t)p.mtiles + mt) * p.s + lane] = keep;
           }
         }
       }
@@ -306,6 +323,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Splits per tile: the smallest S whose units fill the SMs' waves to >= 90%
 // (each split keeps at least 4 K-chunks).
+// u[k][b] = SiLU(sum of the K-split partials + b1[k]) + h[b], stored as the
+// bf16 pair (hi, lo = u - hi) in rows 2b, 2b+1 of stage 2's B operand.
+__global__ void heads_silu_kernel(const float* __restrict__ part, int S, int K, int B, int d,
+                                  const __nv_bfloat16* __restrict__ b1,
+                                  const __nv_bfloat16* __restrict__ h,
+                                  __nv_bfloat16* __restrict__ u) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= K * d) return;
+  const int kh = i / d, m = i - kh * d;
+  const float bias = b1 ? __bfloat162float(b1[i]) : 0.f;
+  for (int b = 0; b < B; ++b) {
+    float a = bias;
+    for (int s2 = 0; s2 < S; ++s2) a += part[(((size_t)s2 * K + kh) * B + b) * d + m];
+    const float uu = a / (1.f + expf(-a)) + __bfloat162float(h[(size_t)b * d + m]);
+    const __nv_bfloat16 hi = __float2bfloat16_rn(uu);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(uu - __bfloat162float(hi));
+    __nv_bfloat16* urow = u + ((size_t)kh * 2 * B + 2 * b) * d + m;
+    urow[0] = hi;
+    urow[d] = lo;
+  }
+}
+
 int choose_splits(int tiles, int kchunks, int sms) {
   int best = 1;
   double best_eff = 0.0;
@@ -341,10 +380,10 @@ TcPlan make_plan(int B, int d, int V, int K, int s) {
   P.S2 = choose_splits(K * P.mt2, P.kch, sms);
   WsCarver w;
   P.off_u = w.take<__nv_bfloat16>((size_t)K * 2 * B * d);
-  P.off_p1 = w.take<float>(P.S1 > 1 ? (size_t)K * P.mt1 * P.S1 * B * BM : 0);
+  P.off_p1 = w.take<float>((size_t)P.S1 * K * B * d);
   P.off_p2 = w.take<float>(P.S2 > 1 ? (size_t)K * P.mt2 * P.S2 * 2 * B * BM : 0);
   P.off_cnt = w.take<int>((size_t)K * (P.mt1 + P.mt2));
-  P.off_cand = w.take<uint64_t>((size_t)B * K * P.mt2 * 4 * s);
+  P.off_cand = w.take<uint64_t>((size_t)B * K * P.mt2 * s);
   P.total = w.total();
   return P;
 }
@@ -440,6 +479,14 @@ int heads_tc_launch(const HeadsArgs& a, cudaStream_t st) {
   p1.counters = counters;
   int rc = dispatch_stage(P.nc1, mA1, mB1, p1, st);
   if (rc) return rc;
+  {
+    const int n = a.K * a.d;
+    heads_silu_kernel<<<(n + 255) / 256, 256, 0, st>>>(p1.part, P.S1, a.K, a.B, a.d,
+                                                     (const __nv_bfloat16*)a.b1,
+                                                     (const __nv_bfloat16*)a.h, u);
+    cudaError_t e2 = cudaGetLastError();
+    if (e2 != cudaSuccess) return cuda_fail(e2, "heads_silu_kernel launch");
+  }
 
   TcParams p2 = p1;
   p2.stage = 2;
@@ -457,7 +504,7 @@ int heads_tc_launch(const HeadsArgs& a, cudaStream_t st) {
   if (rc) return rc;
 
   if (a.topk_idx)
-    return topk_keys_launch(cand, a.B * a.K, P.mt2 * 4 * a.s, a.s, a.topk_idx, a.topk_val, st);
+    return topk_keys_launch(cand, a.B * a.K, P.mt2 * a.s, a.s, a.topk_idx, a.topk_val, st);
   return MEDUSA_OK;
 }
 

@@ -393,7 +393,8 @@ int medusa_tree_attention(const void* q, const void* k_cache, const void* v_cach
     return fail(MEDUSA_ERR_INVALID_ARG, "need Hq % Hkv == 0 and positive head counts");
   if (dh != 64 && dh != 128) return fail(MEDUSA_ERR_UNSUPPORTED, "dh must be 64 or 128");
   if (Lcap < tree->N) return fail(MEDUSA_ERR_INVALID_ARG, "Lcap < N");
-  if (!std::isfinite(scale)) return fail(MEDUSA_ERR_INVALID_ARG, "scale not finite");
+  if (!(std::isfinite(scale) && scale > 0.f))
+    return fail(MEDUSA_ERR_INVALID_ARG, "scale must be finite and > 0");
   if (B == 0) return MEDUSA_OK;
   if (!q || !k_cache || !v_cache || !prefix_len || !out)
     return fail(MEDUSA_ERR_INVALID_ARG, "NULL pointer");

@@ -79,9 +79,17 @@ __global__ void __launch_bounds__(kThreads) topk_keys_kernel(const uint64_t* __r
 #pragma unroll
   for (int i = 0; i < kSmax; ++i) k[i] = 0ull;
   uint64_t kth = 0ull;
-  for (int i = threadIdx.x; i < C; i += kThreads) {
-    const uint64_t key = __ldcg(kr + i);
-    if (key > kth) topk_insert<kSmax>(k, s, key, kth);
+  // 8 independent loads in flight per thread before any insertion
+  for (int base = threadIdx.x; base < C; base += 8 * kThreads) {
+    uint64_t kk[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = base + u * kThreads;
+      kk[u] = i < C ? __ldcg(kr + i) : 0ull;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (kk[u] > kth) topk_insert<kSmax>(k, s, kk[u], kth);
   }
   block_select(k, s, red, idx + row * s, val ? val + row * s : nullptr);
 }
