@@ -180,6 +180,15 @@ int medusa_build_tree(const medusa_tree_t* tree, const int32_t* root_tok,
 size_t medusa_tree_attention_workspace_size(const medusa_tree_t* tree, int B,
                                             int Hq, int Hkv, int dh, int Lcap);
 
+/*
+ * Number of key chunks medusa_tree_attention splits each (sequence, kv-head)
+ * into for these sizes on the current device (>= 1; with more than one, a
+ * combine kernel follows the attention kernel).  Negative status on bad
+ * arguments.  Introspection only (used to count kernel launches).
+ */
+int medusa_tree_attention_chunks(const medusa_tree_t* tree, int B, int Hq,
+                                 int Hkv, int dh, int Lcap, int dtype);
+
 int medusa_tree_attention(const void* q, const void* k_cache,
                           const void* v_cache, const int32_t* prefix_len,
                           const medusa_tree_t* tree, int B, int Hq, int Hkv,

@@ -165,6 +165,13 @@ def attention_workspace_size(tree: Tree, B, Hq, Hkv, dh, Lcap) -> int:
     return int(L.lib().medusa_tree_attention_workspace_size(tree.handle, B, Hq, Hkv, dh, Lcap))
 
 
+def attention_chunks(tree: Tree, B, Hq, Hkv, dh, Lcap, dtype: torch.dtype) -> int:
+    n = int(L.lib().medusa_tree_attention_chunks(tree.handle, B, Hq, Hkv, dh, Lcap, _DT[dtype]))
+    if n < 1:
+        L.check(n, "medusa_tree_attention_chunks")
+    return n
+
+
 def medusa_tree_attention(q, k_cache, v_cache, prefix_len, tree: Tree, scale: float, out=None,
                           ws=None):
     B, N, Hq, dh = q.shape

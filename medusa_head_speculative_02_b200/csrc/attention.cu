@@ -246,6 +246,11 @@ TcPlan make_tc_plan(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lc
 }
 }  // namespace
 
+int attention_chunks(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lcap, int dtype) {
+  if (attention_tc_eligible(dtype, dh, Hq, Hkv)) return make_tc_plan(t, B, Hq, Hkv, dh, Lcap).P;
+  return make_plan(t, B, Hq, Hkv, dh, Lcap).chunks;
+}
+
 size_t attention_workspace(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lcap,
                            int dtype) {
   const size_t simt = make_plan(t, B, Hq, Hkv, dh, Lcap).total;

@@ -89,6 +89,7 @@ struct AttnArgs {
 size_t attention_workspace(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lcap,
                            int dtype);
 int attention_launch(const AttnArgs& a, cudaStream_t st);
+int attention_chunks(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lcap, int dtype);
 // tcgen05 path (bf16, dh = 128, GQA group dividing 128)
 bool attention_tc_eligible(int dtype, int dh, int Hq, int Hkv);
 int attention_tc_chunks(int B, int Hq, int Hkv, int N, int Lcap);

@@ -16,7 +16,9 @@ from . import api
 from .synthetic import MedusaConfig, gen_inputs, plant_verify_logits
 
 # kernels this library launches per call (host memsets excluded)
-LAUNCHES = {"heads": 3, "build_tree": 1, "tree_attention": 2, "accept": 2, "kv_compact": 1}
+# (stage-1 GEMM, SiLU epilogue, stage-2 GEMM, top-s merge; attention adds a
+# combine kernel when it splits the keys into chunks)
+LAUNCHES = {"heads": 4, "build_tree": 1, "tree_attention": 1, "accept": 2, "kv_compact": 1}
 
 
 class VerifyStep:
@@ -95,9 +97,11 @@ class VerifyStep:
         self.compact()
 
     def launches_per_step(self) -> int:
-        n_acc = 2 if self.cfg.accept == "both" else 1
+        c = self.cfg
+        n_acc = 2 if c.accept == "both" else 1
+        chunks = api.attention_chunks(self.tree, c.B, c.Hq, c.Hkv, c.dh, c.Lcap, c.torch_dtype)
         return (LAUNCHES["heads"] + LAUNCHES["build_tree"] + LAUNCHES["tree_attention"] +
-                n_acc * LAUNCHES["accept"] + LAUNCHES["kv_compact"])
+                (1 if chunks > 1 else 0) + n_acc * LAUNCHES["accept"] + LAUNCHES["kv_compact"])
 
     # algorithmic bytes --------------------------------------------------------
     def heads_bytes(self) -> int:
