@@ -6,50 +6,55 @@
 // the cached prefix (slots 0..L_b-1) and to the tree slots L_b + j of the
 // nodes j on its root path (itself included).
 //
-// One CTA = (128 query rows, key chunk, sequence x kv-head).  The query rows
-// of a kv-head are the tree nodes x the GQA group, packed so every K/V tile
-// staged in shared memory serves all of them (the row tiles of one kv-head
-// are adjacent in launch order and share tiles through L2).  Per 128-key
-// tile:
-//   S  = Q K^T        tcgen05.mma, Q and K K-major in smem, S in TMEM
-//                     (double-buffered so S(j+1) overlaps softmax(j))
-//   softmax           8 warps, two threads per query row (64 columns each):
-//                     tcgen05.ld of the S half-row, prefix limit /
-//                     ancestor-bitmask mask, tile max exchanged between the
-//                     halves through TMEM, running max with lazy rescaling
-//                     (the reference max moves only when it grows by more
-//                     than 2^8, then the O row is rescaled in TMEM),
-//                     P = 2^(scale*s - m) as bf16 into a double-buffered,
-//                     128-byte-swizzled K-major smem tile
-//   O += P V          tcgen05.mma, V is the MN-major operand straight from
-//                     its TMA tile, O accumulates in TMEM
-// Warp 0 issues the TMA loads (Q once, a 2-deep ring of K and V tiles),
-// warp 1 issues all MMAs from one thread, warps 2-9 run the softmax and the
-// epilogue.  Warps whose rows are all padding (fewer than 128 query rows)
-// keep the barrier protocol but skip the arithmetic.  With one chunk the CTA
-// writes the normalised output; with more it writes unnormalised partials
-// (O, max, sum) for the combine kernel.
+// Query rows of a (sequence, kv-head) are the tree nodes x the GQA group,
+// packed 128 to an MMA tile.  A CTA takes one 128-row query tile and one key
+// chunk of one (sequence, kv-head).  Per 128-key tile t:
+//   S  = Q K^T        tcgen05.mma (M 128, N 128, K 128): Q and K K-major in
+//                     smem (TMA, 128-byte swizzle), S into TMEM buffer t & 1,
+//                     so the S of tile t+1 is computed while the softmax of
+//                     tile t runs
+//   softmax           two warpgroups, one per 64-key half of the tile; a
+//                     thread owns one query row of one half: one TMEM read of
+//                     its 64 scores, prefix limit / ancestor-bitmask mask, a
+//                     running max per half with lazy rescaling (the
+//                     reference max moves only when it grows by more than
+//                     2^8; the O row is then rescaled in TMEM once the
+//                     previous P.V is done), P = 2^(scale*s - m) with packed
+//                     fp32x2 arithmetic, one pair in four of the exponentials
+//                     on the FMA pipe (polynomial) and the rest on MUFU,
+//                     written as bf16 pairs over the S columns just read
+//   O_h += P_h V_h    tcgen05.mma (M 128, N 128, K 64) per half h: A = P_h
+//                     from TMEM, V_h the MN-major smem operand
+// Each half keeps its own O accumulator and (max, sum); the two states are
+// merged at the end.  TMEM (512 columns): S/P buffers 0 and 1, O_0, O_1, 128
+// columns each.  Warp 0 streams Q and the K ring, warp 10 the V ring (3
+// stages of 128 keys each), warp 1 issues the MMAs, warps 2-5 / 6-9 are the
+// softmax warpgroups of key halves 0 / 1.  With one chunk the CTA writes the
+// normalised output; with more it writes unnormalised partials (O, max, sum)
+// for the combine kernel.
 #include "common.cuh"
 #include "internal.h"
 
 namespace medusa {
 namespace {
 
-constexpr int kThreads = 352;  // K producer, MMA issuer, 8 softmax warps, V producer
+constexpr int kThreads = 352;  // K producer, MMA issuer, 2 x 4 softmax warps, V producer
 constexpr int kVWarp = 10;
-constexpr int BM = 128;  // query rows per CTA
+constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // keys per tile
 constexpr int DH = 128;
-constexpr uint32_t HALF = 128 * 64 * 2;  // one 64-column half of a 128-row bf16 tile
+constexpr uint32_t HALF = 128 * 64 * 2;  // 64-column half of a 128-row bf16 tile: 16 KB
 constexpr uint32_t TILE = 2 * HALF;      // 32 KB
-constexpr int KV_STAGES = 3;
-constexpr size_t SMEM = 1024 + (1 + 2 * KV_STAGES) * (size_t)TILE + 256;  // Q | K[3] | V[3] | barriers
+constexpr int kStages = 3;
+constexpr size_t kDataBytes = (1 + 2 * kStages) * (size_t)TILE;  // Q | K ring | V ring
+constexpr size_t SMEM = 1024 + kDataBytes + 256;
 constexpr float kRescale = 8.0f;  // log2 of the growth that forces a rescale
+static_assert(MEDUSA_MAX_N == 256, "ancestor words are selected for at most 4 x 64 nodes");
 
 struct TcAttnParams {
   const int32_t* L;
   const uint32_t* anc;
-  int B, N, W, Hq, Hkv, G, Lcap, R, P;
+  int B, N, W, Hq, Hkv, G, Lcap, R, P, mtiles;
   float qscale;  // softmax scale * log2(e)
   __nv_bfloat16* out;
   float* po;
@@ -65,7 +70,7 @@ __device__ __forceinline__ Range chunk_range(const TcAttnParams& p, int Lb, int 
   Range rg{0, 0, 0, 0};
   if (!seq_ok) return rg;
   int per = (Lb + p.P - 1) / p.P;
-  per = (per + BN - 1) / BN * BN;
+  per = (per + BN - 1) / BN * BN;  // whole 128-key tiles
   rg.k_lo = min(Lb, chunk * per);
   rg.k_hi = min(Lb, rg.k_lo + per);
   rg.n_pre = (rg.k_hi - rg.k_lo + BN - 1) / BN;
@@ -105,25 +110,24 @@ __device__ __forceinline__ void write_row(const TcAttnParams& p, int b, int kvh,
   }
 }
 
-// Scores of one 64-column half (hf) of tile j with masked columns set to
-// -inf: prefix tiles past the chunk end, tree tiles outside the row's
+// Scores of the 64-key half hf of 128-key tile j with masked columns set to
+// -inf: prefix keys past the chunk end, tree slots outside the row's
 // ancestor set (am = its ancestor bitmask words).
-__device__ __forceinline__ void mask_half(float (&v)[64], int hf, int j, const Range& rg, int N,
+__device__ __forceinline__ void mask_half(float (&v)[64], int j, int hf, const Range& rg, int N,
                                           const uint32_t (&am)[MEDUSA_MAX_N / 32]) {
   if (j < rg.n_pre) {
-    const int lim = rg.k_hi - (rg.k_lo + j * BN) - hf * 64;
+    const int lim = rg.k_hi - (rg.k_lo + j * BN + hf * 64);
     if (lim < 64) {
 #pragma unroll
       for (int c = 0; c < 64; ++c) v[c] = (c < lim) ? v[c] : -INFINITY;
     }
   } else {
-    const int tt = j - rg.n_pre;  // tree tile: nodes tt*128 .. tt*128+127
-    // words of nodes tt*128 + 64*hf .. +63 (tt is 0 or 1 as N <= 256);
-    // selects rather than a run-time index keep am[] in registers
-    const uint32_t a0 = tt ? am[4] : am[0], a1 = tt ? am[5] : am[1];
-    const uint32_t a2 = tt ? am[6] : am[2], a3 = tt ? am[7] : am[3];
-    const uint32_t w0 = hf ? a2 : a0, w1 = hf ? a3 : a1;
-    const int nvalid = N - tt * BN - hf * 64;
+    // nodes 64q .. 64q+63, q < 4 as N <= 256; selects rather than a run-time
+    // index keep am[] in registers
+    const int q = 2 * (j - rg.n_pre) + hf;
+    const uint32_t w0 = q == 0 ? am[0] : q == 1 ? am[2] : q == 2 ? am[4] : am[6];
+    const uint32_t w1 = q == 0 ? am[1] : q == 1 ? am[3] : q == 2 ? am[5] : am[7];
+    const int nvalid = N - q * 64;
 #pragma unroll
     for (int c = 0; c < 64; ++c) {
       const uint32_t word = c < 32 ? w0 : w1;
@@ -149,27 +153,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tmV, const TcAttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+
+  const int qt = blockIdx.x, chunk = blockIdx.y, bk = blockIdx.z;
+  const int b = bk / p.Hkv, kvh = bk - b * p.Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* sQ = sm;
-  uint8_t* sK = sm + TILE;                   // [KV_STAGES]
-  uint8_t* sV = sm + (1 + KV_STAGES) * TILE;  // [KV_STAGES]
-  uint64_t* bars = (uint64_t*)(sm + (1 + 2 * KV_STAGES) * TILE);
+  uint8_t* sK = sm + TILE;
+  uint8_t* sV = sK + kStages * TILE;
+  uint64_t* bars = (uint64_t*)(sm + kDataBytes);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;                    // [KV_STAGES]
-  uint64_t* k_empty = k_full + KV_STAGES;         // [KV_STAGES]
-  uint64_t* v_full = k_empty + KV_STAGES;         // [KV_STAGES]
-  uint64_t* v_empty = v_full + KV_STAGES;         // [KV_STAGES]
-  uint64_t* s_full = v_empty + KV_STAGES;         // [2]
-  uint64_t* s_free = s_full + 2;                  // [2]
-  uint64_t* p_full = s_free + 2;  // softmax wrote P (TMEM)
-  uint64_t* o_done = p_full + 1;  // every P.V completed (P free, O stable)
-  uint64_t* o_final = o_done + 1; // the last P.V completed
-  uint64_t* mma_done = o_final + 1;
+  uint64_t* k_full = bars + 1;              // [kStages]
+  uint64_t* k_empty = k_full + kStages;     // [kStages]
+  uint64_t* v_full = k_empty + kStages;     // [kStages]
+  uint64_t* v_empty = v_full + kStages;     // [kStages]
+  uint64_t* s_full = v_empty + kStages;     // [S/P buffer]
+  uint64_t* p_full = s_full + 2;            // [S/P buffer]
+  uint64_t* pv_done = p_full + 2;           // [S/P buffer]
+  uint64_t* mma_done = pv_done + 2;
   uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
-  const int mt = blockIdx.x, chunk = blockIdx.y, bk = blockIdx.z;
-  const int b = bk / p.Hkv, kvh = bk - b * p.Hkv;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Lb = p.L[b];
   const bool seq_ok = Lb >= 0 && (long long)Lb + p.N <= p.Lcap;
   const Range rg = chunk_range(p, Lb, chunk, seq_ok);
@@ -177,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (T == 0) {  // nothing to attend to in this chunk
     if (threadIdx.x < BM) {
-      const int grow = mt * BM + threadIdx.x;
+      const int grow = qt * BM + threadIdx.x;
       if (grow < p.R) write_row<DH>(p, b, kvh, chunk, grow, 0, -INFINITY, 0.f, nullptr, true);
     }
     return;
@@ -185,7 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < KV_STAGES; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
       mbar_init(&v_full[i], 1);
@@ -193,18 +196,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 256);
+      mbar_init(&p_full[i], 8);  // every softmax warp
+      mbar_init(&pv_done[i], 1);
     }
-    mbar_init(p_full, 8);
-    mbar_init(o_done, 1);
-    mbar_init(o_final, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
     __syncwarp();
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(tmem_slot, 512);  // S/P 0 | S/P 1 | O_0 | O_1
   }
   tc_fence_before();
   __syncthreads();
@@ -213,17 +214,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 || warp == kVWarp) {
     // ---------------------------------------------------------------- TMA producers
-    // warp 0 streams Q and the K tiles, warp 10 the V tiles, so a K tile is
-    // requested as soon as its stage frees (after S), not after the P.V that
-    // frees the V stage of the tile before.
+    // warp 0: the Q tile then the K ring; warp 10: the V ring
     if (lane == 0) {
       const bool isK = warp == 0;
       const uint64_t pol = policy_evict_normal();
       if (isK) {
         prefetch_tmap(&tmQ);
         prefetch_tmap(&tmK);
-        const int zq = b * p.N + mt * (BM / p.G);
         mbar_arrive_expect_tx(q_full, TILE);
+        const int zq = b * p.N + qt * (BM / p.G);
         tma_load_3d(sQ, &tmQ, q_full, 0, kvh * p.G, zq, pol);
         tma_load_3d(sQ + HALF, &tmQ, q_full, 64, kvh * p.G, zq, pol);
       } else {
@@ -235,10 +234,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* buf = isK ? sK : sV;
       int issued = 0;
       for (int j = 0; j < T; ++j) {
-        const int st = j % KV_STAGES;
+        const int st = j % kStages;
         const int key0 = j < rg.n_pre ? rg.k_lo + j * BN : Lb + (j - rg.n_pre) * BN;
         const int z = b * p.Lcap + key0;
-        if (!mbar_wait(&emp[st], ((uint32_t)(j / KV_STAGES) & 1u) ^ 1u, abort_flag)) break;
+        if (!mbar_wait(&emp[st], ((uint32_t)(j / kStages) & 1u) ^ 1u, abort_flag)) break;
         mbar_arrive_expect_tx(&ful[st], TILE);
         tma_load_3d(buf + st * TILE, map, &ful[st], 0, kvh, z, pol);
         tma_load_3d(buf + st * TILE + HALF, map, &ful[st], 64, kvh, z, pol);
@@ -247,191 +246,205 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (issued < T) {
         // aborted: let the loads already issued land before the CTA exits
         if (isK) mbar_wait(q_full, 0u, nullptr);
-        for (int j = (issued > KV_STAGES ? issued - KV_STAGES : 0); j < issued; ++j)
-          mbar_wait(&ful[j % KV_STAGES], (uint32_t)(j / KV_STAGES) & 1u, nullptr);
+        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+          mbar_wait(&ful[j % kStages], (uint32_t)(j / kStages) & 1u, nullptr);
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
+    // S(0), S(1), then for u = 0, 1, ...: P.V(u), S(u + 2) once P.V(u) is
+    // done (S(u+2) reuses the S/P buffer of tile u).
     if (lane == 0) {
       const uint32_t idesc_s = umma_idesc_bf16_f32(BM, BN);
       const uint32_t idesc_o = umma_idesc_bf16_f32_bmn(BM, DH);
-      const uint32_t tO = tmem + 256;
-      const uint32_t tP = tmem + 384;  // P: 64 columns of bf16 pairs
+      // descriptors of the tile bases; a K step adds its byte offset / 16 to
+      // the start-address field (no carry: shared addresses are < 2^18)
+      const uint64_t dq = umma_desc_sw128_kmajor(smem_u32(sQ));
+      auto issue_s = [&](int t) -> bool {
+        const int ks = t % kStages;
+        const int bf = t & 1;
+        if (!mbar_wait(&k_full[ks], (uint32_t)(t / kStages) & 1u, abort_flag)) return false;
+        if (t >= 2 && !mbar_wait(&pv_done[bf], ((uint32_t)(t >> 1) & 1u) ^ 1u, abort_flag))
+          return false;
+        tc_fence_after();
+        const uint64_t dk = umma_desc_sw128_kmajor(smem_u32(sK + ks * TILE));
+        const uint32_t dS = tmem + (uint32_t)bf * 128u;
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint64_t off = (uint64_t)(((kk >> 2) * HALF + (kk & 3) * 32) >> 4);
+          umma_bf16(dS, dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&k_empty[ks]);
+        umma_commit(&s_full[bf]);
+        return true;
+      };
+      auto issue_pv = [&](int u) -> bool {
+        const int vs = u % kStages;
+        const int bf = u & 1;
+        if (!mbar_wait(&p_full[bf], (uint32_t)(u >> 1) & 1u, abort_flag)) return false;
+        if (!mbar_wait(&v_full[vs], (uint32_t)(u / kStages) & 1u, abort_flag)) return false;
+        tc_fence_after();
+        const uint64_t dv = umma_desc_sw128(smem_u32(sV + vs * TILE), HALF, 1024u);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const uint32_t dO = tmem + 256u + (uint32_t)hf * 128u;
+          const uint32_t aP = tmem + (uint32_t)(bf * 128 + hf * 64);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16_ts(dO, aP + (uint32_t)kk * 8u,
+                         dv + (uint64_t)((hf * 64 * 128 + kk * 16 * 128) >> 4), idesc_o,
+                         (u > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&v_empty[vs]);
+        umma_commit(&pv_done[bf]);
+        return true;
+      };
       bool ok = mbar_wait(q_full, 0u, abort_flag);
-      for (int j = 0; j <= T && ok; ++j) {
-        if (j < T) {
-          const int ks = j % KV_STAGES;
-          const int sb = j & 1;  // S buffer
-          if (!mbar_wait(&k_full[ks], (uint32_t)(j / KV_STAGES) & 1u, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(&s_free[sb], ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t tS = tmem + (uint32_t)sb * BN;
-#pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk) {
-            const uint32_t off = (uint32_t)(kk >> 2) * HALF + (uint32_t)(kk & 3) * 32u;
-            umma_bf16(tS, umma_desc_sw128_kmajor(smem_u32(sQ) + off),
-                      umma_desc_sw128_kmajor(smem_u32(sK + ks * TILE) + off), idesc_s,
-                      kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&k_empty[ks]);
-          umma_commit(&s_full[sb]);
-        }
-        if (j >= 1) {
-          // O += P V with P (bf16, written by the softmax warps) read from TMEM
-          const int jj = j - 1;
-          const int vs = jj % KV_STAGES;
-          if (!mbar_wait(p_full, (uint32_t)(jj & 1), abort_flag)) { ok = false; break; }
-          if (!mbar_wait(&v_full[vs], (uint32_t)(jj / KV_STAGES) & 1u, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            umma_bf16_ts(tO, tP + (uint32_t)kk * 8u,
-                         umma_desc_sw128(smem_u32(sV + vs * TILE) + (uint32_t)kk * 2048u, HALF,
-                                         1024u),
-                         idesc_o, (jj > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&v_empty[vs]);
-          umma_commit(o_done);
-          if (jj == T - 1) umma_commit(o_final);
-        }
+      if (ok) ok = issue_s(0);
+      if (ok && T > 1) ok = issue_s(1);
+      for (int u = 0; u < T && ok; ++u) {
+        ok = issue_pv(u);
+        if (ok && u + 2 < T) ok = issue_s(u + 2);
       }
       umma_commit(mma_done);
       mbar_wait(mma_done, 0u, nullptr);
     }
   } else {
-    // ---------------------------------------------------------------- softmax + epilogue
-    // Two warpgroups share every S row: warps 2-5 take columns 0-63, warps
-    // 6-9 columns 64-127 (two warps per SM sub-partition for latency
-    // hiding).  The halves exchange their tile maxima and final sums through
-    // spare TMEM columns (384 + ...), as the row's two threads sit in
-    // different warps of the same TMEM lane quadrant.
-    const int half = warp >= 6 ? 1 : 0;
-    const int cb = half * 64;
-    const int q4 = warp & 3;
+    // ---------------------------------------------------------------- softmax warpgroups
+    const int hf = (warp - 2) >> 2;  // key half of every tile
+    const int q4 = warp & 3;         // TMEM lane quadrant of this warp
     const int r = q4 * 32 + lane;
-    const int grow = mt * BM + r;
+    const int grow = qt * BM + r;
     const bool row_ok = grow < p.R;
-    const bool warp_live = (mt * BM + q4 * 32) < p.R;  // warp-uniform
+    const bool warp_live = (qt * BM + q4 * 32) < p.R;  // warp-uniform
     const int node = min(grow / p.G, p.N - 1);
     uint32_t am[MEDUSA_MAX_N / 32];
 #pragma unroll
     for (int w = 0; w < MEDUSA_MAX_N / 32; ++w) am[w] = (w < p.W) ? p.anc[(size_t)node * p.W + w] : 0u;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-    const uint32_t tx = tmem + lane_base + 448;  // exchange columns
+    const uint32_t tO = tmem + lane_base + 256u + (uint32_t)hf * 128u;
+    const unsigned long long q2 = f2_pack(p.qscale, p.qscale);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < T; ++j) {
-      const int st = j & 1;
-      bool good = ok && mbar_wait(&s_full[st], (j >> 1) & 1u, abort_flag);
+    for (int t = 0; t < T; ++t) {
+      const int bf = t & 1;
+      const uint32_t tS = tmem + lane_base + (uint32_t)(bf * 128 + hf * 64);
+      const bool good = mbar_wait(&s_full[bf], (uint32_t)(t >> 1) & 1u, abort_flag);
       if (!__all_sync(0xffffffffu, good)) {
-        // no named barrier inside this loop: every wait is bounded, so the
-        // other warps leave as soon as their own waits see the abort flag
-        ok = false;
+        ok = false;  // every wait is bounded: the other warps leave on the abort flag
         break;
       }
       tc_fence_after();
       if (!warp_live) {
-        // every row of this warp is padding past the last query row: keep
-        // the barrier protocol, skip the arithmetic (its P rows are never
-        // output; O rows are independent of each other).  Waiting for
-        // PV(j-1) first keeps this arrival out of tile j-1's phase.
-        tc_fence_before();
-        mbar_arrive(&s_free[st]);
-        if (j >= 1) {
-          const bool w_ok = mbar_wait(o_done, (uint32_t)((j - 1) & 1), abort_flag);
-          if (!__all_sync(0xffffffffu, w_ok)) { ok = false; continue; }
-        }
+        // rows past the last query row: keep the protocol, skip the work
+        // (O rows are independent of each other, these are never output)
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
+        if (lane == 0) mbar_arrive(&p_full[bf]);
         continue;
       }
-      // the whole row's max: the other half is read too (instead of trading
-      // maxima with the other warpgroup), so the two halves never wait for
-      // each other within a tile and their MUFU phases can drift apart
-      float s[64];
-      float omax;
-      {
-        float t[64];
-        tmem_ld64(tmem + lane_base + (uint32_t)st * BN + (uint32_t)(64 - cb), t);
-        mask_half(t, half ^ 1, j, rg, p.N, am);
-        omax = max64(t);
-      }
-      tmem_ld64(tmem + lane_base + (uint32_t)st * BN + (uint32_t)cb, s);
-      tc_fence_before();
-      mbar_arrive(&s_free[st]);
-      mask_half(s, half, j, rg, p.N, am);
-      const float hmax = max64(s);
-      const float tmax = fmaxf(hmax, omax) * p.qscale;  // scale > 0
-      float corr = 1.f;
-      bool rescale = false;
-      if (tmax > m_used + kRescale) {
-        corr = ex2_approx(m_used - tmax);  // 0 when m_used is -inf
-        m_used = tmax;
-        l *= corr;
-        rescale = true;
-      }
-      // p = 2^(scale*s - m); a row with no visible key yet has m = -inf and
-      // only -inf scores, for which 2^(-inf) = 0 with any finite offset
-      const float moff = (m_used == -INFINITY) ? 0.f : m_used;
-      float sum8[8];
+      float v[64];
+      tmem_ld64(tS, v);
+      mask_half(v, t, hf, rg, p.N, am);
+      const float tmax = max64(v) * p.qscale;  // scale > 0
+      const bool grow_m = tmax > m_used + kRescale;
+      // warp-uniform branch: the TMEM accesses and the vote are collective
+      if (__any_sync(0xffffffffu, grow_m)) {
+        float corr = 1.f;
+        if (grow_m) {
+          corr = ex2_approx(m_used - tmax);  // 0 when m_used is -inf
+          m_used = tmax;
+          l *= corr;
+        }
+        if (t > 0) {
+          // O must hold every P.V so far: wait for P.V(t-1)
+          const bool w_ok = mbar_wait(&pv_done[(t - 1) & 1], (uint32_t)((t - 1) >> 1) & 1u, abort_flag);
+          if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll
-      for (int e = 0; e < 8; ++e) sum8[e] = 0.f;
+          for (int c0 = 0; c0 < DH; c0 += 16) {
+            float o16[16];
+            tmem_ld16(tO + c0, o16);
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float e = ex2_approx(fmaf(s[c], p.qscale, -moff));
-        s[c] = e;
-        sum8[c & 7] += e;
-      }
-      l += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
-
-      // P (TMEM) is free and O stable once PV(j-1) has completed; PV(j-2)
-      // completed before this softmax's previous tile went on, so o_done is
-      // at most one completion away from the awaited one
-      if (j >= 1) {
-        const bool w_ok = mbar_wait(o_done, (uint32_t)((j - 1) & 1), abort_flag);
-        if (!__all_sync(0xffffffffu, w_ok)) { ok = false; continue; }
-        tc_fence_after();
-        // each half rescales its own 64 columns of the O row
-        if (__any_sync(0xffffffffu, rescale)) {
-          const uint32_t tO = tmem + lane_base + 256 + (uint32_t)cb;
-#pragma unroll
-          for (int c0 = 0; c0 < 64; c0 += 16) {
-            float t[16];
-            tmem_ld16(tO + c0, t);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) t[e] *= corr;
-            tmem_st16(tO + c0, t);
+            for (int e = 0; e < 16; ++e) o16[e] *= corr;
+            tmem_st16(tO + c0, o16);
           }
         }
       }
-      // my 64 keys of the P row -> TMEM columns 384 + 32*half, bf16 pairs
-      {
-        uint32_t pk[32];
+      // P = 2^(scale*s - m) in packed pairs (a row with no visible key yet
+      // has m = -inf and only -inf scores, whose exponentials are zeroed)
+      const float moff = (m_used == -INFINITY) ? 0.f : m_used;
+      const unsigned long long m2 = f2_pack(-moff, -moff);
+      unsigned long long sum2[4] = {0ull, 0ull, 0ull, 0ull};
+      uint32_t pk[32];
 #pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) pk[c2] = pack_bf16x2_pos(s[2 * c2], s[2 * c2 + 1]);
-        tmem_st32(tmem + lane_base + 384u + (uint32_t)(half * 32), pk);
+      for (int c2 = 0; c2 < 32; ++c2) {
+        float x0, x1, e0, e1;
+        f2_unpack(f2_fma(f2_pack(v[2 * c2], v[2 * c2 + 1]), q2, m2), x0, x1);
+        if ((c2 & 3) == 3) {
+          exp2_fma2(x0, x1, e0, e1);
+          e0 = (v[2 * c2] == -INFINITY) ? 0.f : e0;
+          e1 = (v[2 * c2 + 1] == -INFINITY) ? 0.f : e1;
+        } else {
+          e0 = ex2_approx(x0);
+          e1 = ex2_approx(x1);
+        }
+        sum2[c2 & 3] = f2_add(sum2[c2 & 3], f2_pack(e0, e1));
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
+        pk[c2] = *reinterpret_cast<const uint32_t*>(&h2);
+      }
+      tmem_st32(tS, pk);  // P over the S columns just read
+      {
+        float a0, a1, b0, b1, c0f, c1f, d0, d1;
+        f2_unpack(sum2[0], a0, a1);
+        f2_unpack(sum2[1], b0, b1);
+        f2_unpack(sum2[2], c0f, c1f);
+        f2_unpack(sum2[3], d0, d1);
+        l += ((a0 + a1) + (b0 + b1)) + ((c0f + c1f) + (d0 + d1));
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[bf]);
     }
-    // combine the halves' sums, then the epilogue (every softmax thread
-    // reaches this barrier: the loop above leaves only all together)
+    // last P.V complete (it commits after every earlier MMA)
     if (ok && warp_live) {
-      tmem_st1(tx + 4u + (uint32_t)half, l);
+      const bool good = mbar_wait(&pv_done[(T - 1) & 1], (uint32_t)((T - 1) >> 1) & 1u, abort_flag);
+      ok = __all_sync(0xffffffffu, good);
+    }
+    // merge the two halves' states: each publishes (m, l) in columns 2hf,
+    // 2hf+1 of S/P buffer 0 (free now), then finishes 64 of the 128 output
+    // columns from both O accumulators
+    if (ok && warp_live) {
+      tmem_st1(tmem + lane_base + (uint32_t)(2 * hf), m_used);
+      tmem_st1(tmem + lane_base + (uint32_t)(2 * hf + 1), l);
       tc_fence_before();
     }
     const bool bad = bar_red_or(2, 256, !ok || *abort_flag);
     if (!bad && warp_live) {
       tc_fence_after();
-      l += tmem_ld1(tx + 4u + (uint32_t)(half ^ 1));
-      bool w_ok = mbar_wait(o_final, 0u, abort_flag);
-      w_ok = __all_sync(0xffffffffu, w_ok);
-      if (w_ok) {
-        tc_fence_after();
-        float o[64];
-        tmem_ld64(tmem + lane_base + 256 + (uint32_t)cb, o);
-        if (row_ok) write_row<64>(p, b, kvh, chunk, grow, cb, m_used, l, o, half == 0);
+      const uint32_t tX = tmem + lane_base + (uint32_t)(2 * (hf ^ 1));
+      const float m_x = tmem_ld1(tX), l_x = tmem_ld1(tX + 1u);
+      const float m0 = hf ? m_x : m_used, l0 = hf ? l_x : l;
+      const float m1 = hf ? m_used : m_x, l1 = hf ? l : l_x;
+      const float M = fmaxf(m0, m1);
+      const float w0 = (m0 == -INFINITY) ? 0.f : ex2_approx(m0 - M);
+      const float w1 = (m1 == -INFINITY) ? 0.f : ex2_approx(m1 - M);
+      const float Ls = w0 * l0 + w1 * l1;
+      const uint32_t tO0 = tmem + lane_base + 256u, tO1 = tO0 + 128u;
+      const int cb = hf * 64;
+#pragma unroll
+      for (int c0 = 0; c0 < 64; c0 += 32) {
+        float a[32], bb[32];
+        tmem_ld32(tO0 + (uint32_t)(cb + c0), a);
+        tmem_ld32(tO1 + (uint32_t)(cb + c0), bb);
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          a[e] = (w0 != 0.f ? w0 * a[e] : 0.f) + (w1 != 0.f ? w1 * bb[e] : 0.f);
+        if (row_ok) {
+          if (M == -INFINITY)
+            write_row<32>(p, b, kvh, chunk, grow, cb + c0, M, Ls, nullptr, hf == 0 && c0 == 0);
+          else
+            write_row<32>(p, b, kvh, chunk, grow, cb + c0, M, Ls, a, hf == 0 && c0 == 0);
+        }
       }
     }
   }
@@ -457,8 +470,8 @@ int attention_tc_chunks(int B, int Hq, int Hkv, int N, int Lcap) {
   const long long R = (long long)N * G;
   const long long units = (long long)B * Hkv * ((R + BM - 1) / BM);
   const int sms = num_sms();
-  long long P = (3LL * sms + units - 1) / units;
-  const long long max_p = ((long long)(Lcap - N) + 2 * BN - 1) / (2 * BN);  // >= 2 tiles each
+  long long P = (2LL * sms + units - 1) / units;
+  const long long max_p = ((long long)(Lcap - N) + 4 * BN - 1) / (4 * BN);  // >= 4 tiles each
   if (P > max_p) P = max_p;
   if (P < 1) P = 1;
   return (int)P;
@@ -480,7 +493,7 @@ int attention_tc_run(const AttnArgs& a, int P, float* po, float2* pml, cudaStrea
   {
     const uint64_t dims[3] = {(uint64_t)DH, (uint64_t)a.Hkv, (uint64_t)a.B * a.Lcap};
     const uint64_t strides[2] = {(uint64_t)DH * 2, (uint64_t)a.Hkv * DH * 2};
-    const uint32_t box[3] = {64, 1, BN};
+    const uint32_t box[3] = {64, 1, BN};  // 64 dh x 1 head x 128 keys
     int rc = make_tmap_bf16(&mK, a.k, 3, dims, strides, box);
     if (rc) return rc;
     rc = make_tmap_bf16(&mV, a.v, 3, dims, strides, box);
@@ -507,6 +520,7 @@ int attention_tc_run(const AttnArgs& a, int P, float* po, float2* pml, cudaStrea
   p.Lcap = a.Lcap;
   p.R = R;
   p.P = P;
+  p.mtiles = mtiles;
   p.qscale = a.scale * 1.4426950408889634f;
   p.out = (__nv_bfloat16*)a.out;
   p.po = po;

@@ -116,6 +116,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0u;
 }
+// try_wait with an explicit suspend-time limit (ns): a suspended thread
+// resumes as soon as the phase completes, or after the limit.
+__device__ __forceinline__ bool mbar_try_wait_for(uint64_t* bar, uint32_t parity,
+                                                  uint32_t limit_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(limit_ns)
+      : "memory");
+  return ok != 0u;
+}
 // Bounded wait for phase `parity` of `bar`.  Returns false (and raises the
 // device status word and the CTA's abort flag) if it ran out, or if another
 // role of the CTA already aborted.
@@ -123,15 +137,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0u) {
-      if (abort_flag != nullptr && *abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        atomicOr(&g_dev_status, DEV_TIMEOUT);
-        if (abort_flag != nullptr) *abort_flag = 1;
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_for(bar, parity, 200000u)) return true;
+    if (abort_flag != nullptr && *abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(&g_dev_status, DEV_TIMEOUT);
+      if (abort_flag != nullptr) *abort_flag = 1;
+      return false;
     }
   }
 }
@@ -389,6 +401,56 @@ __device__ __forceinline__ float exp2_fma(float x) {
   const float p = fmaf(fmaf(fmaf(0.05517166853f, f, 0.24261112511f), f, 0.69326096773f), f,
                        0.99992805719f);
   return __int_as_float(__float_as_int(p) + (n << 23));
+}
+// Non-blocking test of phase `parity` of `bar`.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0u;
+}
+// Packed fp32 pairs (Blackwell f32x2 FMA / ADD): a 64-bit register holds
+// (lo, hi).
+__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(unsigned long long r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// Two 2^x on the FMA pipe in packed form (same method as exp2_fma).
+__device__ __forceinline__ void exp2_fma2(float x0, float x1, float& e0, float& e1) {
+  const unsigned long long x2 = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const unsigned long long t2 = f2_add(x2, f2_pack(12582912.0f, 12582912.0f));
+  const unsigned long long f2 = f2_add(x2, f2_add(t2, f2_pack(-12582912.0f, -12582912.0f)) ^
+                                               0x8000000080000000ull);
+  const unsigned long long p2 =
+      f2_fma(f2_fma(f2_fma(f2_pack(0.05517166853f, 0.05517166853f), f2,
+                           f2_pack(0.24261112511f, 0.24261112511f)),
+                    f2, f2_pack(0.69326096773f, 0.69326096773f)),
+             f2, f2_pack(0.99992805719f, 0.99992805719f));
+  float t0, t1, p0, p1;
+  f2_unpack(t2, t0, t1);
+  f2_unpack(p2, p0, p1);
+  e0 = __int_as_float(__float_as_int(p0) + ((__float_as_int(t0) - 0x4B400000) << 23));
+  e1 = __int_as_float(__float_as_int(p1) + ((__float_as_int(t1) - 0x4B400000) << 23));
 }
 // Two non-negative floats to a bf16x2 word (first argument in the low half),
 // rounding half up, with integer ops only (no conversion-pipe instruction).
