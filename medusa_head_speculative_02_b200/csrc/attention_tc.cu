@@ -9,29 +9,29 @@
 // Query rows of a (sequence, kv-head) are the tree nodes x the GQA group,
 // packed 128 to an MMA tile.  A CTA takes one 128-row query tile and one key
 // chunk of one (sequence, kv-head).  Per 128-key tile t:
-//   S  = Q K^T        tcgen05.mma (M 128, N 128, K 128): Q and K K-major in
-//                     smem (TMA, 128-byte swizzle), S into TMEM buffer t & 1,
-//                     so the S of tile t+1 is computed while the softmax of
-//                     tile t runs
-//   softmax           two warpgroups, one per 64-key half of the tile; a
-//                     thread owns one query row of one half: one TMEM read of
-//                     its 64 scores, prefix limit / ancestor-bitmask mask, a
-//                     running max per half with lazy rescaling (the
-//                     reference max moves only when it grows by more than
-//                     2^8; the O row is then rescaled in TMEM once the
-//                     previous P.V is done), P = 2^(scale*s - m) with packed
-//                     fp32x2 arithmetic, one pair in four of the exponentials
-//                     on the FMA pipe (polynomial) and the rest on MUFU,
-//                     written as bf16 pairs over the S columns just read
-//   O_h += P_h V_h    tcgen05.mma (M 128, N 128, K 64) per half h: A = P_h
-//                     from TMEM, V_h the MN-major smem operand
-// Each half keeps its own O accumulator and (max, sum); the two states are
-// merged at the end.  TMEM (512 columns): S/P buffers 0 and 1, O_0, O_1, 128
-// columns each.  Warp 0 streams Q and the K ring, warp 10 the V ring (3
-// stages of 128 keys each), warp 1 issues the MMAs, warps 2-5 / 6-9 are the
-// softmax warpgroups of key halves 0 / 1.  With one chunk the CTA writes the
-// normalised output; with more it writes unnormalised partials (O, max, sum)
-// for the combine kernel.
+//   S  = Q K^T      tcgen05.mma (M 128, N 128, K 128): Q and K K-major in
+//                   smem (TMA, 128-byte swizzle), S into TMEM buffer t mod 3,
+//                   issued while the softmax of tile t-1 runs
+//   softmax         two warpgroups, one per 64-key half of the tile; a thread
+//                   owns one query row of one half: one TMEM read of its 64
+//                   scores, prefix limit / ancestor-bitmask mask, the row max
+//                   of the tile from both halves (exchanged through TMEM),
+//                   one running max per row with lazy rescaling (the
+//                   reference max moves only when it grows by more than 2^8;
+//                   the O row is then rescaled in TMEM once the previous P.V
+//                   is done), P = 2^(scale*s - m) with packed fp32x2
+//                   arithmetic, one pair in four of the exponentials on the
+//                   FMA pipe (polynomial) and the rest on MUFU, written as
+//                   bf16 pairs over the S columns just read
+//   O += P V        tcgen05.mma (M 128, N 128, K 128): A = P from TMEM, V
+//                   the MN-major smem operand
+// TMEM (512 columns): three S/P buffers and O, 128 columns each.  Warp 0
+// streams Q and the K ring, warp 10 the V ring (3 stages of 128 keys each),
+// warp 1 issues the MMAs, warps 2-5 / 6-9 are the softmax warpgroups of key
+// halves 0 / 1; the two warps that share a TMEM lane quadrant meet at a
+// named barrier once per tile.  With one chunk the CTA writes the
+// normalised output; with more it writes unnormalised partials (O, max,
+// sum) for the combine kernel.
 #include "common.cuh"
 #include "internal.h"
 
@@ -167,9 +167,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_full = k_empty + kStages;     // [kStages]
   uint64_t* v_empty = v_full + kStages;     // [kStages]
   uint64_t* s_full = v_empty + kStages;     // [S/P buffer]
-  uint64_t* p_full = s_full + 2;            // [S/P buffer]
-  uint64_t* pv_done = p_full + 2;           // [S/P buffer]
-  uint64_t* mma_done = pv_done + 2;
+  uint64_t* p_full = s_full + 3;            // [S/P buffer]
+  uint64_t* pv_done = p_full + 3;           // [S/P buffer]
+  uint64_t* mma_done = pv_done + 3;
   uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 3; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 8);  // every softmax warp
       mbar_init(&pv_done[i], 1);
@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0) {
     __syncwarp();
-    tmem_alloc(tmem_slot, 512);  // S/P 0 | S/P 1 | O_0 | O_1
+    tmem_alloc(tmem_slot, 512);  // S/P 0 | S/P 1 | S/P 2 | O
   }
   tc_fence_before();
   __syncthreads();
@@ -252,19 +252,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    // S(0), S(1), then for u = 0, 1, ...: P.V(u), S(u + 2) once P.V(u) is
-    // done (S(u+2) reuses the S/P buffer of tile u).
+    // S(0), S(1), then for u = 0, 1, ...: P.V(u), S(u + 2).  S(u+2) reuses
+    // the S/P buffer of tile u-1, whose P.V was issued one step earlier and
+    // has normally completed by then, so the tensor pipe is not left idle
+    // waiting for a completion; S still runs a tile ahead of the softmax.
     if (lane == 0) {
       const uint32_t idesc_s = umma_idesc_bf16_f32(BM, BN);
       const uint32_t idesc_o = umma_idesc_bf16_f32_bmn(BM, DH);
       // descriptors of the tile bases; a K step adds its byte offset / 16 to
       // the start-address field (no carry: shared addresses are < 2^18)
       const uint64_t dq = umma_desc_sw128_kmajor(smem_u32(sQ));
+      const uint32_t tOacc = tmem + 384u;
       auto issue_s = [&](int t) -> bool {
         const int ks = t % kStages;
-        const int bf = t & 1;
+        const int bf = t % 3;
         if (!mbar_wait(&k_full[ks], (uint32_t)(t / kStages) & 1u, abort_flag)) return false;
-        if (t >= 2 && !mbar_wait(&pv_done[bf], ((uint32_t)(t >> 1) & 1u) ^ 1u, abort_flag))
+        if (t >= 3 && !mbar_wait(&pv_done[bf], ((uint32_t)(t / 3) & 1u) ^ 1u, abort_flag))
           return false;
         tc_fence_after();
         const uint64_t dk = umma_desc_sw128_kmajor(smem_u32(sK + ks * TILE));
@@ -280,28 +283,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto issue_pv = [&](int u) -> bool {
         const int vs = u % kStages;
-        const int bf = u & 1;
-        if (!mbar_wait(&p_full[bf], (uint32_t)(u >> 1) & 1u, abort_flag)) return false;
+        const int bf = u % 3;
+        if (!mbar_wait(&p_full[bf], (uint32_t)(u / 3) & 1u, abort_flag)) return false;
         if (!mbar_wait(&v_full[vs], (uint32_t)(u / kStages) & 1u, abort_flag)) return false;
         tc_fence_after();
         const uint64_t dv = umma_desc_sw128(smem_u32(sV + vs * TILE), HALF, 1024u);
+        const uint32_t aP = tmem + (uint32_t)bf * 128u;
+        // keys 64 hf + 16 kk .. : P columns 32 hf + 8 kk of the buffer
+        // (column c of a half holds keys 2c, 2c+1), V rows 64 hf + 16 kk
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const uint32_t dO = tmem + 256u + (uint32_t)hf * 128u;
-          const uint32_t aP = tmem + (uint32_t)(bf * 128 + hf * 64);
+        for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_bf16_ts(dO, aP + (uint32_t)kk * 8u,
+            umma_bf16_ts(tOacc, aP + (uint32_t)(hf * 64 + kk * 8),
                          dv + (uint64_t)((hf * 64 * 128 + kk * 16 * 128) >> 4), idesc_o,
-                         (u > 0 || kk > 0) ? 1u : 0u);
-        }
+                         (u > 0 || hf > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&v_empty[vs]);
         umma_commit(&pv_done[bf]);
         return true;
       };
       bool ok = mbar_wait(q_full, 0u, abort_flag);
-      if (ok) ok = issue_s(0);
-      if (ok && T > 1) ok = issue_s(1);
+      for (int t = 0; t < 2 && t < T && ok; ++t) ok = issue_s(t);
       for (int u = 0; u < T && ok; ++u) {
         ok = issue_pv(u);
         if (ok && u + 2 < T) ok = issue_s(u + 2);
@@ -312,29 +314,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------------------------------------------------------- softmax warpgroups
     const int hf = (warp - 2) >> 2;  // key half of every tile
-    const int q4 = warp & 3;         // TMEM lane quadrant of this warp
+    const int q4 = warp & 3;         // TMEM lane quadrant of this warp (shared with its partner)
     const int r = q4 * 32 + lane;
     const int grow = qt * BM + r;
     const bool row_ok = grow < p.R;
-    const bool warp_live = (qt * BM + q4 * 32) < p.R;  // warp-uniform
+    const bool warp_live = (qt * BM + q4 * 32) < p.R;  // warp-uniform, same for both partners
     const int node = min(grow / p.G, p.N - 1);
     uint32_t am[MEDUSA_MAX_N / 32];
 #pragma unroll
     for (int w = 0; w < MEDUSA_MAX_N / 32; ++w) am[w] = (w < p.W) ? p.anc[(size_t)node * p.W + w] : 0u;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-    const uint32_t tO = tmem + lane_base + 256u + (uint32_t)hf * 128u;
+    const uint32_t tO = tmem + lane_base + 384u + (uint32_t)hf * 64u;  // this half's O columns
     const unsigned long long q2 = f2_pack(p.qscale, p.qscale);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
+    // Every exit from the tile loop follows a pair barrier whose result is
+    // the OR of both partners' error flags, so neither is left waiting.
+    bool err = false;
     for (int t = 0; t < T; ++t) {
-      const int bf = t & 1;
+      const int bf = t % 3;
       const uint32_t tS = tmem + lane_base + (uint32_t)(bf * 128 + hf * 64);
-      const bool good = mbar_wait(&s_full[bf], (uint32_t)(t >> 1) & 1u, abort_flag);
-      if (!__all_sync(0xffffffffu, good)) {
-        ok = false;  // every wait is bounded: the other warps leave on the abort flag
+      const bool good = mbar_wait(&s_full[bf], (uint32_t)(t / 3) & 1u, abort_flag);
+      err = err || !__all_sync(0xffffffffu, good);
+      float v[64];
+      float tmax = -INFINITY;
+      if (!err && warp_live) {
+        tc_fence_after();
+        tmem_ld64(tS, v);
+        mask_half(v, t, hf, rg, p.N, am);
+        tmax = max64(v) * p.qscale;  // scale > 0
+        tmem_st1(tS + 32u, tmax);   // column 32 of the half is not overwritten by P
+        tc_fence_before();
+      }
+      if (bar_red_or(3 + q4, 64, err)) {
+        ok = false;
         break;
       }
-      tc_fence_after();
       if (!warp_live) {
         // rows past the last query row: keep the protocol, skip the work
         // (O rows are independent of each other, these are never output)
@@ -342,11 +357,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&p_full[bf]);
         continue;
       }
-      float v[64];
-      tmem_ld64(tS, v);
-      mask_half(v, t, hf, rg, p.N, am);
-      const float tmax = max64(v) * p.qscale;  // scale > 0
-      const bool grow_m = tmax > m_used + kRescale;
+      tc_fence_after();
+      tmax = fmaxf(tmax, tmem_ld1(tmem + lane_base + (uint32_t)(bf * 128 + (hf ^ 1) * 64 + 32)));
+      const bool grow_m = tmax > m_used + kRescale;  // the same in both partners
       // warp-uniform branch: the TMEM accesses and the vote are collective
       if (__any_sync(0xffffffffu, grow_m)) {
         float corr = 1.f;
@@ -357,16 +370,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (t > 0) {
           // O must hold every P.V so far: wait for P.V(t-1)
-          const bool w_ok = mbar_wait(&pv_done[(t - 1) & 1], (uint32_t)((t - 1) >> 1) & 1u, abort_flag);
-          if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
-          tc_fence_after();
+          const bool w_ok = mbar_wait(&pv_done[(t - 1) % 3], (uint32_t)((t - 1) / 3) & 1u, abort_flag);
+          if (__all_sync(0xffffffffu, w_ok)) {
+            tc_fence_after();
 #pragma unroll
-          for (int c0 = 0; c0 < DH; c0 += 16) {
-            float o16[16];
-            tmem_ld16(tO + c0, o16);
+            for (int c0 = 0; c0 < 64; c0 += 16) {
+              float o16[16];
+              tmem_ld16(tO + c0, o16);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) o16[e] *= corr;
-            tmem_st16(tO + c0, o16);
+              for (int e = 0; e < 16; ++e) o16[e] *= corr;
+              tmem_st16(tO + c0, o16);
+            }
+          } else {
+            err = true;  // reported at the next pair barrier (or the final one)
           }
         }
       }
@@ -405,45 +421,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[bf]);
     }
+    ok = ok && !err;
     // last P.V complete (it commits after every earlier MMA)
     if (ok && warp_live) {
-      const bool good = mbar_wait(&pv_done[(T - 1) & 1], (uint32_t)((T - 1) >> 1) & 1u, abort_flag);
+      const bool good = mbar_wait(&pv_done[(T - 1) % 3], (uint32_t)((T - 1) / 3) & 1u, abort_flag);
       ok = __all_sync(0xffffffffu, good);
     }
-    // merge the two halves' states: each publishes (m, l) in columns 2hf,
-    // 2hf+1 of S/P buffer 0 (free now), then finishes 64 of the 128 output
-    // columns from both O accumulators
+    // row sum = both halves' partial sums: each publishes its own in column
+    // hf of S/P buffer 0 (free now), then finishes its 64 output columns
     if (ok && warp_live) {
-      tmem_st1(tmem + lane_base + (uint32_t)(2 * hf), m_used);
-      tmem_st1(tmem + lane_base + (uint32_t)(2 * hf + 1), l);
+      tmem_st1(tmem + lane_base + (uint32_t)hf, l);
       tc_fence_before();
     }
     const bool bad = bar_red_or(2, 256, !ok || *abort_flag);
     if (!bad && warp_live) {
       tc_fence_after();
-      const uint32_t tX = tmem + lane_base + (uint32_t)(2 * (hf ^ 1));
-      const float m_x = tmem_ld1(tX), l_x = tmem_ld1(tX + 1u);
-      const float m0 = hf ? m_x : m_used, l0 = hf ? l_x : l;
-      const float m1 = hf ? m_used : m_x, l1 = hf ? l : l_x;
-      const float M = fmaxf(m0, m1);
-      const float w0 = (m0 == -INFINITY) ? 0.f : ex2_approx(m0 - M);
-      const float w1 = (m1 == -INFINITY) ? 0.f : ex2_approx(m1 - M);
-      const float Ls = w0 * l0 + w1 * l1;
-      const uint32_t tO0 = tmem + lane_base + 256u, tO1 = tO0 + 128u;
+      const float Ls = l + tmem_ld1(tmem + lane_base + (uint32_t)(hf ^ 1));
       const int cb = hf * 64;
 #pragma unroll
       for (int c0 = 0; c0 < 64; c0 += 32) {
-        float a[32], bb[32];
-        tmem_ld32(tO0 + (uint32_t)(cb + c0), a);
-        tmem_ld32(tO1 + (uint32_t)(cb + c0), bb);
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          a[e] = (w0 != 0.f ? w0 * a[e] : 0.f) + (w1 != 0.f ? w1 * bb[e] : 0.f);
+        float a[32];
+        tmem_ld32(tO + (uint32_t)c0, a);
         if (row_ok) {
-          if (M == -INFINITY)
-            write_row<32>(p, b, kvh, chunk, grow, cb + c0, M, Ls, nullptr, hf == 0 && c0 == 0);
+          if (m_used == -INFINITY)
+            write_row<32>(p, b, kvh, chunk, grow, cb + c0, m_used, Ls, nullptr, hf == 0 && c0 == 0);
           else
-            write_row<32>(p, b, kvh, chunk, grow, cb + c0, M, Ls, a, hf == 0 && c0 == 0);
+            write_row<32>(p, b, kvh, chunk, grow, cb + c0, m_used, Ls, a, hf == 0 && c0 == 0);
         }
       }
     }
