@@ -12,8 +12,13 @@
 // desc, index asc) and, for typical acceptance, the base-2 online softmax
 // statistics of z = l * log2(e) / T:  m = max z, Z = sum 2^(z-m),
 // S = sum 2^(z-m) (z-m).  Natural-log entropy: H = ln Z - ln2 * S / Z.
-// Phase 2 (accept_walk_kernel, one warp per sequence): merge the chunks of
-// the N rows, decide every node's own condition against its parent row,
+// A thread folds one 16-byte load at a time: one max per load, the first
+// index recomputed only when that max improves, and the softmax statistics
+// rescaled at most once per load.  -inf logits add nothing; NaN logits are
+// outside the contract (they never win the argmax and add nothing).
+// Phase 2 (accept_walk_kernel, one CTA per sequence, one thread per node):
+// merge the chunks of the N rows, decide every node's own condition against
+// its parent row,
 // accept a node iff its whole root path satisfies the condition (ancestor
 // bitmask test), take the deepest accepted node (ties: lowest index) and
 // emit its path and the argmax of its row.
@@ -38,25 +43,6 @@ struct Soft {
   float m, Z, S;
 };
 
-__device__ __forceinline__ void soft_add(Soft& a, float z) {
-  if (a.Z == 0.f) {
-    a.m = z;
-    a.Z = 1.f;
-    a.S = 0.f;
-  } else if (z <= a.m) {
-    const float t = z - a.m;
-    const float e = exp2f(t);
-    a.Z += e;
-    a.S = fmaf(e, t, a.S);
-  } else {
-    const float t = a.m - z;  // < 0
-    const float c = exp2f(t);
-    a.S = c * fmaf(t, a.Z, a.S);
-    a.Z = fmaf(c, a.Z, 1.f);
-    a.m = z;
-  }
-}
-
 __device__ __forceinline__ Soft soft_merge(Soft a, Soft b) {
   if (b.Z == 0.f) return a;
   if (a.Z == 0.f) return b;
@@ -70,41 +56,118 @@ __device__ __forceinline__ Soft soft_merge(Soft a, Soft b) {
   return r;
 }
 
+// Eight bf16 or four fp32 logits of one 16-byte load, as floats.
+template <typename T> struct Lanes;
+template <> struct Lanes<__nv_bfloat16> {
+  static constexpr int n = 8;
+  static __device__ __forceinline__ void get(const uint4& w, float (&x)[8]) {
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[2 * i] = __uint_as_float(u[i] << 16);
+      x[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
+    }
+  }
+};
+template <> struct Lanes<float> {
+  static constexpr int n = 4;
+  static __device__ __forceinline__ void get(const uint4& w, float (&x)[4]) {
+    x[0] = __uint_as_float(w.x);
+    x[1] = __uint_as_float(w.y);
+    x[2] = __uint_as_float(w.z);
+    x[3] = __uint_as_float(w.w);
+  }
+};
+
+// Running per-thread state of the row reduction: the argmax (value, first
+// index) and, for typical acceptance, (m, Z, S) of z = x * zscale in base 2.
+struct RedState {
+  float bv;
+  int bi;
+  Soft sf;
+};
+
+// Folds NV consecutive logits starting at column `base` (indices increase
+// from call to call within a thread, so a strict > keeps the first maximum).
+template <bool TYPICAL, int NV>
+__device__ __forceinline__ void red_consume(RedState& st, const float (&x)[NV], int base,
+                                            float zscale) {
+  float vm = x[0];
+#pragma unroll
+  for (int j = 1; j < NV; ++j) vm = fmaxf(vm, x[j]);
+  if (vm > st.bv) {
+    int jj = NV - 1;
+#pragma unroll
+    for (int j = NV - 1; j >= 0; --j) jj = (x[j] == vm) ? j : jj;
+    st.bv = vm;
+    st.bi = base + jj;
+  }
+  if (TYPICAL) {
+    const float vz = vm * zscale;  // zscale > 0: the max of the scaled values
+    if (vz > st.sf.m) {
+      if (st.sf.Z > 0.f) {
+        const float d = st.sf.m - vz;  // < 0
+        const float c = ex2_approx(d);
+        st.sf.S = c * fmaf(d, st.sf.Z, st.sf.S);
+        st.sf.Z *= c;
+      }
+      st.sf.m = vz;
+    }
+    if (st.sf.m != -INFINITY) {  // else every value so far is -inf: nothing to add
+#pragma unroll
+      for (int j = 0; j < NV; ++j) {
+        // t <= 0; clamped so that a -inf (or NaN) logit adds 0 to Z and S
+        const float t = fmaxf(fmaf(x[j], zscale, -st.sf.m), -200.f);
+        const float e = ex2_approx(t);
+        st.sf.Z += e;
+        st.sf.S = fmaf(e, t, st.sf.S);
+      }
+    }
+  }
+}
+
 template <typename T, bool TYPICAL>
 __global__ void __launch_bounds__(kRedThreads)
     row_reduce_kernel(const T* __restrict__ vlog, int V, int chunk, int splits, float zscale,
                       RowPart* __restrict__ parts) {
+  // nothing in this kernel runs ahead of its predecessor
+  griddep_launch_dependents();
+  griddep_wait();
   const size_t row = blockIdx.x;
   const int sp = blockIdx.y;
   const int lo = sp * chunk;
   const int hi = min(V, lo + chunk);
   const T* xr = vlog + row * (size_t)V;
-  uint64_t best = 0ull;
-  Soft sf{-INFINITY, 0.f, 0.f};
-  constexpr int VEC = 16 / sizeof(T);
+  constexpr int VEC = Lanes<T>::n;
+  RedState st{-INFINITY, 0x7FFFFFFF, Soft{-INFINITY, 0.f, 0.f}};
   const bool vec_ok = ((((uintptr_t)(xr + lo)) & 15u) == 0) && ((hi - lo) % VEC == 0);
   if (vec_ok) {
     const uint4* p = reinterpret_cast<const uint4*>(xr + lo);
     const int nv = (hi - lo) / VEC;
-    for (int i = threadIdx.x; i < nv; i += kRedThreads) {
-      const uint4 w = __ldcs(p + i);
-      const T* e = reinterpret_cast<const T*>(&w);
-#pragma unroll
-      for (int j = 0; j < VEC; ++j) {
-        const float x = to_f32(e[j]);
-        const uint64_t key = make_key(x, (uint32_t)(lo + i * VEC + j));
-        best = key > best ? key : best;
-        if (TYPICAL) soft_add(sf, x * zscale);
+    // a thread whose values are all -inf reports its first column
+    if ((int)threadIdx.x < nv) st.bi = lo + (int)threadIdx.x * VEC;
+    // two 16-byte loads in flight per thread
+    for (int i = threadIdx.x; i < nv; i += 2 * kRedThreads) {
+      const bool two = i + kRedThreads < nv;
+      const uint4 w0 = __ldcs(p + i);
+      const uint4 w1 = two ? __ldcs(p + i + kRedThreads) : make_uint4(0u, 0u, 0u, 0u);
+      float x[VEC];
+      Lanes<T>::get(w0, x);
+      red_consume<TYPICAL, VEC>(st, x, lo + i * VEC, zscale);
+      if (two) {
+        Lanes<T>::get(w1, x);
+        red_consume<TYPICAL, VEC>(st, x, lo + (i + kRedThreads) * VEC, zscale);
       }
     }
   } else {
+    if (lo + (int)threadIdx.x < hi) st.bi = lo + (int)threadIdx.x;
     for (int i = lo + threadIdx.x; i < hi; i += kRedThreads) {
-      const float x = to_f32(xr[i]);
-      const uint64_t key = make_key(x, (uint32_t)i);
-      best = key > best ? key : best;
-      if (TYPICAL) soft_add(sf, x * zscale);
+      const float x[1] = {to_f32(xr[i])};
+      red_consume<TYPICAL, 1>(st, x, i, zscale);
     }
   }
+  uint64_t best = make_key(st.bv, (uint32_t)st.bi);
+  Soft sf = st.sf;
   // block reduction
   best = warp_max_u64(best);
   if (TYPICAL) {
@@ -140,21 +203,29 @@ __global__ void __launch_bounds__(kRedThreads)
   }
 }
 
+// One CTA per sequence, one thread per tree node (blockDim = N rounded up to
+// a whole warp, <= MEDUSA_MAX_N).
 template <typename T, bool TYPICAL>
-__global__ void __launch_bounds__(32)
+__global__ void __launch_bounds__(MEDUSA_MAX_N)
     accept_walk_kernel(const T* __restrict__ vlog, const RowPart* __restrict__ parts, int splits,
                        const int32_t* __restrict__ tok, const int32_t* __restrict__ parent,
                        const int32_t* __restrict__ depth, const uint32_t* __restrict__ anc, int N,
                        int W, int K, int V, float zscale, float eps, float delta,
                        int32_t* __restrict__ accept_len, int32_t* __restrict__ accept_nodes,
                        int32_t* __restrict__ next_tok) {
+  // nothing in this kernel runs ahead of its predecessor
+  griddep_launch_dependents();
+  griddep_wait();
   __shared__ int32_t amax[MEDUSA_MAX_N];
   __shared__ float mrow[MEDUSA_MAX_N], zrow[MEDUSA_MAX_N], thr[MEDUSA_MAX_N];
   __shared__ uint32_t cond[MEDUSA_MAX_N / 32];
+  __shared__ uint32_t wkey[MEDUSA_MAX_N / 32];
   const int b = blockIdx.x;
-  const int lane = threadIdx.x;
+  const int n = threadIdx.x;
+  const int warp = n >> 5, lane = n & 31;
 
-  for (int n = lane; n < N; n += 32) {
+  // merge the chunks of row n: argmax and (typical) the acceptance threshold
+  if (n < N) {
     const RowPart* pr = parts + ((size_t)b * N + n) * splits;
     uint64_t best = 0ull;
     Soft sf{-INFINITY, 0.f, 0.f};
@@ -171,57 +242,54 @@ __global__ void __launch_bounds__(32)
       thr[n] = fminf(eps, delta * expf(-H));
     }
   }
-  __syncwarp();
+  __syncthreads();
 
-  // each node's own condition (root: true)
-  for (int n0 = 0; n0 < N; n0 += 32) {
-    const int n = n0 + lane;
-    bool c = (n == 0);
-    if (n > 0 && n < N) {
-      const int par = parent[n];
-      const int t = tok[(size_t)b * N + n];
-      if (TYPICAL) {
-        if (t >= 0 && t < V) {
-          const float x = to_f32(vlog[((size_t)b * N + par) * V + t]);
-          const float p = exp2f(x * zscale - mrow[par]) / zrow[par];
-          c = p > thr[par];
-        }
-      } else {
-        c = (amax[par] == t);
+  // node n's own condition against its parent's row (root: true)
+  bool c = (n == 0);
+  if (n > 0 && n < N) {
+    const int par = parent[n];
+    const int t = tok[(size_t)b * N + n];
+    if (TYPICAL) {
+      if (t >= 0 && t < V) {
+        const float x = to_f32(vlog[((size_t)b * N + par) * V + t]);
+        const float p = exp2f(x * zscale - mrow[par]) / zrow[par];
+        c = p > thr[par];
       }
+    } else {
+      c = (amax[par] == t);
     }
-    const uint32_t bits = __ballot_sync(0xffffffffu, c);
-    if (lane == 0) cond[n0 >> 5] = bits;
   }
-  __syncwarp();
+  const uint32_t bits = __ballot_sync(0xffffffffu, c);
+  if (lane == 0) cond[warp] = bits;
+  __syncthreads();
 
   // accepted iff every node on the root path satisfies its condition;
   // deepest accepted node wins, ties to the lowest index.
   uint32_t key = 0u;
-  for (int n = lane; n < N; n += 32) {
+  if (n < N) {
     bool ok = true;
     for (int w = 0; w < W; ++w) ok = ok && ((anc[(size_t)n * W + w] & ~cond[w]) == 0u);
-    if (ok) {
-      const uint32_t k2 = ((uint32_t)depth[n] << 16) | (0xFFFFu - (uint32_t)n);
-      key = k2 > key ? k2 : key;
-    }
+    if (ok) key = ((uint32_t)depth[n] << 16) | (0xFFFFu - (uint32_t)n);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const uint32_t other = __shfl_xor_sync(0xffffffffu, key, o);
     key = other > key ? other : key;
   }
-  const int best = (int)(0xFFFFu - (key & 0xFFFFu));
-  const int D = (int)(key >> 16);
-  if (lane == 0) {
+  if (lane == 0) wkey[warp] = key;
+  __syncthreads();
+  if (n == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) key = wkey[w] > key ? wkey[w] : key;
+    const int best = (int)(0xFFFFu - (key & 0xFFFFu));
+    const int D = (int)(key >> 16);
     accept_len[b] = D;
     next_tok[b] = amax[best];
     int j = 0;
     for (int w = 0; w < W; ++w) {
-      uint32_t bits = anc[(size_t)best * W + w];
-      while (bits) {
-        const int i = __ffs(bits) - 1;
-        bits &= bits - 1;
+      uint32_t bitsw = anc[(size_t)best * W + w];
+      while (bitsw) {
+        const int i = __ffs(bitsw) - 1;
+        bitsw &= bitsw - 1;
         if (j <= K) accept_nodes[(size_t)b * (K + 1) + j] = w * 32 + i;
         ++j;
       }
@@ -268,14 +336,18 @@ int accept_launch(const AcceptArgs& a, cudaStream_t st) {
   RowPart* parts = (RowPart*)a.ws;
   const float zscale = a.typical ? kLog2e / a.temperature : 0.f;
   dim3 g1(rows, P.splits);
+  const int walk_threads = (N + 31) / 32 * 32;
   const medusa_tree* t = a.tree;
-#define MEDUSA_ACC(T, TYP)                                                                    \
-  do {                                                                                        \
-    row_reduce_kernel<T, TYP><<<g1, kRedThreads, 0, st>>>((const T*)a.vlog, a.V, P.chunk,     \
-                                                          P.splits, zscale, parts);           \
-    accept_walk_kernel<T, TYP><<<a.B, 32, 0, st>>>(                                           \
-        (const T*)a.vlog, parts, P.splits, a.tok, t->d_parent, t->d_depth, t->d_anc, N, t->W, \
-        t->K, a.V, zscale, a.eps, a.delta, a.accept_len, a.accept_nodes, a.next_tok);         \
+  cudaError_t le = cudaSuccess;
+#define MEDUSA_ACC(T, TYP)                                                                     \
+  do {                                                                                         \
+    le = launch_pdl(row_reduce_kernel<T, TYP>, g1, dim3(kRedThreads), 0, st, (const T*)a.vlog, \
+                    a.V, P.chunk, P.splits, zscale, parts);                                    \
+    if (le == cudaSuccess)                                                                     \
+      le = launch_pdl(accept_walk_kernel<T, TYP>, dim3(a.B), dim3(walk_threads), 0, st,        \
+                      (const T*)a.vlog, parts, P.splits, a.tok, t->d_parent, t->d_depth,       \
+                      t->d_anc, N, t->W, t->K, a.V, zscale, a.eps, a.delta, a.accept_len,      \
+                      a.accept_nodes, a.next_tok);                                             \
   } while (0)
   if (a.dtype == MEDUSA_F32) {
     if (a.typical) MEDUSA_ACC(float, true);
@@ -285,7 +357,7 @@ int accept_launch(const AcceptArgs& a, cudaStream_t st) {
     else MEDUSA_ACC(__nv_bfloat16, false);
   }
 #undef MEDUSA_ACC
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = le != cudaSuccess ? le : cudaGetLastError();
   return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "accept kernels launch");
 }
 
@@ -345,20 +417,24 @@ int accept_greedy_noalloc_launch(const void* vlog, int dtype, const int32_t* tok
   int rc = scratch_address(&parts);
   if (rc) return rc;
   dim3 g1((unsigned)rows, P.splits);
-#define MEDUSA_ACC_STATIC(T)                                                                    \
-  do {                                                                                          \
-    row_reduce_kernel<T, false><<<g1, kRedThreads, 0, st>>>((const T*)vlog, V, P.chunk,         \
-                                                            P.splits, 0.f, parts);              \
-    accept_walk_kernel<T, false><<<B, 32, 0, st>>>(                                             \
-        (const T*)vlog, parts, P.splits, tok, t->d_parent, t->d_depth, t->d_anc, N, t->W, t->K, \
-        V, 0.f, 0.f, 0.f, accept_len, accept_nodes, next_tok);                                  \
+  const int walk_threads = (N + 31) / 32 * 32;
+  cudaError_t le = cudaSuccess;
+#define MEDUSA_ACC_STATIC(T)                                                                     \
+  do {                                                                                           \
+    le = launch_pdl(row_reduce_kernel<T, false>, g1, dim3(kRedThreads), 0, st, (const T*)vlog, V, \
+                    P.chunk, P.splits, 0.f, parts);                                              \
+    if (le == cudaSuccess)                                                                       \
+      le = launch_pdl(accept_walk_kernel<T, false>, dim3(B), dim3(walk_threads), 0, st,          \
+                      (const T*)vlog,                                                            \
+                      parts, P.splits, tok, t->d_parent, t->d_depth, t->d_anc, N, t->W, t->K, V, \
+                      0.f, 0.f, 0.f, accept_len, accept_nodes, next_tok);                        \
   } while (0)
   if (dtype == MEDUSA_F32)
     MEDUSA_ACC_STATIC(float);
   else
     MEDUSA_ACC_STATIC(__nv_bfloat16);
 #undef MEDUSA_ACC_STATIC
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = le != cudaSuccess ? le : cudaGetLastError();
   return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "accept kernels launch (static scratch)");
 }
 

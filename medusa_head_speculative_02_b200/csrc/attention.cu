@@ -62,6 +62,9 @@ __global__ void __launch_bounds__(kThreads)
                           const uint32_t* __restrict__ anc, int N, int W, int Hq, int Hkv,
                           int Lcap, float qscale, int P, int R, float* __restrict__ po,
                           float2* __restrict__ pml) {
+  // nothing in this kernel runs ahead of its predecessor
+  griddep_launch_dependents();
+  griddep_wait();
   __shared__ float qs[RB][DH];
   __shared__ float ks[TK][DH + 1];
   __shared__ float vs[TK][DH];
@@ -193,6 +196,9 @@ __global__ void tree_attn_combine_kernel(const float* __restrict__ po,
                                          const int32_t* __restrict__ Lp, int B, int N, int Hq,
                                          int Hkv, int Lcap, int chunks, int R,
                                          T* __restrict__ out) {
+  // nothing in this kernel runs ahead of its predecessor
+  griddep_launch_dependents();
+  griddep_wait();
   const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (gw >= B * N * Hq) return;
@@ -274,9 +280,10 @@ int attention_launch(const AttnArgs& a, cudaStream_t st) {
     if (rc || P.P == 1) return rc;
     const int R = t->N * (a.Hq / a.Hkv);
     const int rows = a.B * t->N * a.Hq;
-    tree_attn_combine_kernel<__nv_bfloat16, 128><<<(rows + 7) / 8, 256, 0, st>>>(
-        po, pml, a.L, a.B, t->N, a.Hq, a.Hkv, a.Lcap, P.P, R, (__nv_bfloat16*)a.out);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(tree_attn_combine_kernel<__nv_bfloat16, 128>, dim3((rows + 7) / 8),
+                               dim3(256), 0, st, po, pml, a.L, a.B, t->N, a.Hq, a.Hkv, a.Lcap,
+                               P.P, R, (__nv_bfloat16*)a.out);
+    if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "tree attention combine launch");
   }
   const AttnPlan P = make_plan(t, a.B, a.Hq, a.Hkv, a.dh, a.Lcap);
@@ -289,14 +296,15 @@ int attention_launch(const AttnArgs& a, cudaStream_t st) {
   dim3 g1(P.rblocks, P.chunks, a.B * a.Hkv);
   const int rows = a.B * t->N * a.Hq;
   const int cblocks = (rows + 7) / 8;
+  cudaError_t le = cudaSuccess;
 #define MEDUSA_ATT(T, DH)                                                                        \
   do {                                                                                           \
-    tree_attn_simt_kernel<T, DH><<<g1, kThreads, 0, st>>>(                                       \
-        (const T*)a.q, (const T*)a.k, (const T*)a.v, a.L, t->d_anc, t->N, t->W, a.Hq, a.Hkv,     \
-        a.Lcap, qscale, P.P, P.R, po, pml);                                                      \
-    tree_attn_combine_kernel<T, DH><<<cblocks, 256, 0, st>>>(po, pml, a.L, a.B, t->N, a.Hq,      \
-                                                             a.Hkv, a.Lcap, P.chunks, P.R,       \
-                                                             (T*)a.out);                         \
+    le = launch_pdl(tree_attn_simt_kernel<T, DH>, g1, dim3(kThreads), 0, st, (const T*)a.q,      \
+                    (const T*)a.k, (const T*)a.v, a.L, t->d_anc, t->N, t->W, a.Hq, a.Hkv, a.Lcap, \
+                    qscale, P.P, P.R, po, pml);                                                  \
+    if (le == cudaSuccess)                                                                       \
+      le = launch_pdl(tree_attn_combine_kernel<T, DH>, dim3(cblocks), dim3(256), 0, st, po, pml, \
+                      a.L, a.B, t->N, a.Hq, a.Hkv, a.Lcap, P.chunks, P.R, (T*)a.out);            \
   } while (0)
   if (a.dtype == MEDUSA_F32) {
     if (a.dh == 64) MEDUSA_ATT(float, 64);
@@ -306,7 +314,7 @@ int attention_launch(const AttnArgs& a, cudaStream_t st) {
     else MEDUSA_ATT(__nv_bfloat16, 128);
   }
 #undef MEDUSA_ATT
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = le != cudaSuccess ? le : cudaGetLastError();
   return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "tree attention launch");
 }
 

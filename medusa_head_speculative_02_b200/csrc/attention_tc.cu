@@ -154,6 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
 
+  griddep_wait();  // prefix lengths and the K/V cache may come from the kernel ahead
   const int qt = blockIdx.x, chunk = blockIdx.y, bk = blockIdx.z;
   const int b = bk / p.Hkv, kvh = bk - b * p.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -211,6 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_launch_dependents();  // TMEM taken: the next kernel may be scheduled
 
   if (warp == 0 || warp == kVWarp) {
     // ---------------------------------------------------------------- TMA producers
@@ -529,8 +531,8 @@ int attention_tc_run(const AttnArgs& a, int P, float* po, float2* pml, cudaStrea
   p.po = po;
   p.pml = pml;
   dim3 grid(mtiles, P, a.B * a.Hkv);
-  tree_attn_tc_kernel<<<grid, kThreads, SMEM, st>>>(mQ, mK, mV, p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(tree_attn_tc_kernel, grid, dim3(kThreads), SMEM, st, mQ, mK, mV, p);
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "tree_attn_tc_kernel launch");
 }
 

@@ -496,6 +496,13 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr, uint32_t
 __host__ __device__ constexpr uint32_t umma_idesc_bf16_f32_bmn(int M, int N) {
   return umma_idesc_bf16_f32(M, N) | (1u << 16);
 }
+// Programmatic dependent launch: wait until every kernel this one depends on
+// has completed and its memory is visible; let the next kernel in the stream
+// be scheduled (it still waits in its own griddepcontrol.wait).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 // Orders this thread's generic-proxy shared-memory writes before later
 // async-proxy reads (tensor-core operands).
 __device__ __forceinline__ void fence_proxy_async_smem() {

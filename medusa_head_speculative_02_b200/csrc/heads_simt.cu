@@ -28,6 +28,9 @@ __global__ void __launch_bounds__(kWarps * 32)
                       size_t x_stride_k, const float* __restrict__ b1,
                       const float* __restrict__ h, float* __restrict__ out, int B, int d,
                       int rows_per_head, int K) {
+  // nothing in this kernel runs ahead of its predecessor
+  griddep_launch_dependents();
+  griddep_wait();
   const int gw = blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (gw >= K * rows_per_head) return;
@@ -90,12 +93,15 @@ int heads_simt_launch(const HeadsArgs& a, cudaStream_t st) {
   float* u = (float*)(ws + P.off_u);
   float* logits = a.logits ? a.logits : (float*)(ws + P.off_logits);
   const int rows1 = a.K * a.d, rows2 = a.K * a.V;
-  heads_simt_kernel<<<(rows1 + kWarps - 1) / kWarps, kWarps * 32, 0, st>>>(
-      1, (const float*)a.W1, (const float*)a.h, 0, (const float*)a.b1, (const float*)a.h, u,
-      a.B, a.d, a.d, a.K);
-  heads_simt_kernel<<<(rows2 + kWarps - 1) / kWarps, kWarps * 32, 0, st>>>(
-      2, (const float*)a.W2, u, (size_t)a.B * a.d, nullptr, nullptr, logits, a.B, a.d, a.V, a.K);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(heads_simt_kernel, dim3((rows1 + kWarps - 1) / kWarps),
+                             dim3(kWarps * 32), 0, st, 1, (const float*)a.W1, (const float*)a.h,
+                             (size_t)0, (const float*)a.b1, (const float*)a.h, u, a.B, a.d, a.d,
+                             a.K);
+  if (e == cudaSuccess)
+    e = launch_pdl(heads_simt_kernel, dim3((rows2 + kWarps - 1) / kWarps), dim3(kWarps * 32), 0, st,
+                   2, (const float*)a.W2, (const float*)u, (size_t)a.B * a.d,
+                   (const float*)nullptr, (const float*)nullptr, logits, a.B, a.d, a.V, a.K);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "heads_simt_kernel launch");
   if (a.topk_idx)
     return topk_rows_launch(logits, MEDUSA_F32, a.B * a.K, a.V, a.s, a.topk_idx, a.topk_val, st);

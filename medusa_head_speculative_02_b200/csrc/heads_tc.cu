@@ -132,12 +132,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_launch_dependents();  // TMEM taken: the next kernel may be scheduled
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
+      // The weight tiles of the first STAGES loads depend on no earlier
+      // kernel: they are issued before waiting for the predecessor (whose
+      // output is the activation operand), so the ring fills while it ends.
+      uint32_t pre = 0;
+      for (int unit = blockIdx.x; unit < p.units && pre < (uint32_t)C::STAGES; unit += gridDim.x) {
+        int tile, sp, kh, mt, k0, k1;
+        unit_coords(p, unit, tile, sp, kh, mt, k0, k1);
+        const int row0 = kh * p.rows + mt * BM;
+        for (int kc = k0; kc < k1 && pre < (uint32_t)C::STAGES; ++kc, ++pre) {
+          mbar_arrive_expect_tx(&full[pre], C::STAGE_BYTES);
+          tma_load_2d(sA + (size_t)pre * A_BYTES, &tmA, &full[pre], kc * BK, row0, pol_w);
+        }
+      }
+      griddep_wait();
       uint32_t it = 0;
       bool ok = true;
       for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x) {
@@ -147,12 +162,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kc = k0; kc < k1; ++kc, ++it) {
           const int st = (int)(it % C::STAGES);
           const uint32_t ph = (it / C::STAGES) & 1u;
-          if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag)) {
-            ok = false;
-            break;
+          if (it >= pre) {  // the first `pre` weight tiles are already on their way
+            if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
+            tma_load_2d(sA + (size_t)st * A_BYTES, &tmA, &full[st], kc * BK, row0, pol_w);
           }
-          mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
-          tma_load_2d(sA + (size_t)st * A_BYTES, &tmA, &full[st], kc * BK, row0, pol_w);
           if (p.stage == 1)
             tma_load_2d(sB + (size_t)st * C::B_BYTES, &tmB, &full[st], kc * BK, 0, pol_x);
           else
@@ -325,11 +342,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 // (each split keeps at least 4 K-chunks).
 // u[k][b] = SiLU(sum of the K-split partials + b1[k]) + h[b], stored as the
 // bf16 pair (hi, lo = u - hi) in rows 2b, 2b+1 of stage 2's B operand.
+// It also zeroes the split counters of stage 2, which runs next.
 __global__ void heads_silu_kernel(const float* __restrict__ part, int S, int K, int B, int d,
                                   const __nv_bfloat16* __restrict__ b1,
                                   const __nv_bfloat16* __restrict__ h,
-                                  __nv_bfloat16* __restrict__ u) {
+                                  __nv_bfloat16* __restrict__ u, int* __restrict__ cnt2,
+                                  int ncnt2) {
+  griddep_launch_dependents();  // stage 2 may start streaming its weights
+  griddep_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  for (int j = i; j < ncnt2; j += gridDim.x * blockDim.x) cnt2[j] = 0;
   if (i >= K * d) return;
   const int kh = i / d, m = i - kh * d;
   const float bias = b1 ? __bfloat162float(b1[i]) : 0.f;
@@ -345,14 +367,14 @@ __global__ void heads_silu_kernel(const float* __restrict__ part, int S, int K, 
   }
 }
 
-int choose_splits(int tiles, int kchunks, int sms) {
+int choose_splits(int tiles, int kchunks, int sms, double want) {
   int best = 1;
   double best_eff = 0.0;
   for (int S = 1; S <= 16 && S <= kchunks / 4 + (S == 1); ++S) {
     const long long units = (long long)tiles * S;
     const long long waves = (units + sms - 1) / sms;
     const double eff = (double)units / (double)(waves * sms);
-    if (eff >= 0.9) return S;
+    if (eff >= want) return S;
     if (eff > best_eff + 1e-9) {
       best_eff = eff;
       best = S;
@@ -376,8 +398,8 @@ TcPlan make_plan(int B, int d, int V, int K, int s) {
   P.mt1 = (d + BM - 1) / BM;
   P.mt2 = (V + BM - 1) / BM;
   P.kch = (d + BK - 1) / BK;
-  P.S1 = choose_splits(K * P.mt1, P.kch, sms);
-  P.S2 = choose_splits(K * P.mt2, P.kch, sms);
+  P.S1 = choose_splits(K * P.mt1, P.kch, sms, 0.9);
+  P.S2 = choose_splits(K * P.mt2, P.kch, sms, 0.9);
   WsCarver w;
   P.off_u = w.take<__nv_bfloat16>((size_t)K * 2 * B * d);
   P.off_p1 = w.take<float>((size_t)P.S1 * K * B * d);
@@ -402,8 +424,8 @@ int launch_stage(const CUtensorMap& A, const CUtensorMap& Bm, const TcParams& p,
     attr_set[dev] = true;
   }
   const int grid = p.units < num_sms() ? p.units : num_sms();
-  heads_tc_kernel<NC><<<grid, kThreads, C::SMEM, st>>>(A, Bm, p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(heads_tc_kernel<NC>, dim3(grid), dim3(kThreads), C::SMEM, st, A, Bm, p);
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "heads_tc_kernel launch");
 }
 
@@ -458,9 +480,6 @@ int heads_tc_launch(const HeadsArgs& a, cudaStream_t st) {
     if (rc) return rc;
   }
 
-  cudaError_t e = cudaMemsetAsync(counters, 0, sizeof(int) * (size_t)a.K * (P.mt1 + P.mt2), st);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(heads counters)");
-
   TcParams p1{};
   p1.stage = 1;
   p1.K = a.K;
@@ -481,10 +500,11 @@ int heads_tc_launch(const HeadsArgs& a, cudaStream_t st) {
   if (rc) return rc;
   {
     const int n = a.K * a.d;
-    heads_silu_kernel<<<(n + 255) / 256, 256, 0, st>>>(p1.part, P.S1, a.K, a.B, a.d,
-                                                     (const __nv_bfloat16*)a.b1,
-                                                     (const __nv_bfloat16*)a.h, u);
-    cudaError_t e2 = cudaGetLastError();
+    cudaError_t e2 = launch_pdl(heads_silu_kernel, dim3((n + 255) / 256), dim3(256), 0, st, p1.part,
+                                P.S1, a.K, a.B, a.d, (const __nv_bfloat16*)a.b1,
+                                (const __nv_bfloat16*)a.h, u, counters + (size_t)a.K * P.mt1,
+                                a.K * P.mt2);
+    if (e2 == cudaSuccess) e2 = cudaGetLastError();
     if (e2 != cudaSuccess) return cuda_fail(e2, "heads_silu_kernel launch");
   }
 

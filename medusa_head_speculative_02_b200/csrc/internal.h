@@ -30,6 +30,30 @@ int fail(int code, const std::string& msg);
 int cuda_fail(cudaError_t e, const char* what);
 int num_sms();
 
+// Launches a kernel of this library with programmatic stream serialization:
+// it may be scheduled before the kernel ahead of it in the stream has
+// finished, once every CTA of that kernel has signalled
+// griddepcontrol.launch_dependents (or exited).  Every kernel launched this
+// way executes griddepcontrol.wait before its first access to memory that
+// another kernel of the library writes, and signals its dependents only
+// after taking its TMEM, so a waiting CTA never holds resources its
+// predecessor still needs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Carves 256-byte-aligned segments out of a caller workspace.
 struct WsCarver {
   size_t off = 0;

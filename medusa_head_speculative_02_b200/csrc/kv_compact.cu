@@ -20,6 +20,9 @@ __global__ void kv_compact_kernel(VecT* __restrict__ kc, VecT* __restrict__ vc,
                                   const int32_t* __restrict__ alen,
                                   const int32_t* __restrict__ anodes, int Lcap, int K,
                                   size_t slot_vecs, int32_t* __restrict__ new_len) {
+  // nothing in this kernel runs ahead of its predecessor
+  griddep_launch_dependents();
+  griddep_wait();
   const int b = blockIdx.y;
   const size_t x = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int a = alen[b];
@@ -47,18 +50,19 @@ int kv_compact_launch(void* k, void* v, const int32_t* L, const int32_t* alen,
   const size_t esize = dtype == MEDUSA_F32 ? 4 : 2;
   const size_t slot_bytes = (size_t)Hkv * dh * esize;
   const bool v16 = (slot_bytes % 16 == 0) && ((((uintptr_t)k) | ((uintptr_t)v)) % 16 == 0);
+  cudaError_t e;
   if (v16) {
     const size_t nv = slot_bytes / 16;
     dim3 grid((unsigned)((nv + 127) / 128), B);
-    kv_compact_kernel<uint4><<<grid, 128, 0, st>>>((uint4*)k, (uint4*)v, L, alen, anodes, Lcap,
-                                                   K, nv, new_len);
+    e = launch_pdl(kv_compact_kernel<uint4>, grid, dim3(128), 0, st, (uint4*)k, (uint4*)v, L, alen,
+                   anodes, Lcap, K, nv, new_len);
   } else {
     const size_t nv = slot_bytes / 4;
     dim3 grid((unsigned)((nv + 127) / 128), B);
-    kv_compact_kernel<uint32_t><<<grid, 128, 0, st>>>((uint32_t*)k, (uint32_t*)v, L, alen,
-                                                      anodes, Lcap, K, nv, new_len);
+    e = launch_pdl(kv_compact_kernel<uint32_t>, grid, dim3(128), 0, st, (uint32_t*)k, (uint32_t*)v,
+                   L, alen, anodes, Lcap, K, nv, new_len);
   }
-  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "kv_compact_kernel launch");
 }
 

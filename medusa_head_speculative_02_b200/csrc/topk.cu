@@ -39,6 +39,9 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) topk_rows_kernel(const T* __restrict__ x, int V, int s,
                                                              int32_t* __restrict__ idx,
                                                              float* __restrict__ val) {
+  // nothing in this kernel runs ahead of its predecessor
+  griddep_launch_dependents();
+  griddep_wait();
   __shared__ uint64_t red[kThreads / 32];
   const size_t row = blockIdx.x;
   const T* xr = x + row * (size_t)V;
@@ -72,6 +75,9 @@ __global__ void __launch_bounds__(kThreads) topk_keys_kernel(const uint64_t* __r
                                                              int C, int s,
                                                              int32_t* __restrict__ idx,
                                                              float* __restrict__ val) {
+  // nothing in this kernel runs ahead of its predecessor
+  griddep_launch_dependents();
+  griddep_wait();
   __shared__ uint64_t red[kThreads / 32];
   const size_t row = blockIdx.x;
   const uint64_t* kr = keys + row * (size_t)C;
@@ -99,20 +105,22 @@ __global__ void __launch_bounds__(kThreads) topk_keys_kernel(const uint64_t* __r
 int topk_rows_launch(const void* x, int dtype, int R, int V, int s, int32_t* idx, float* val,
                      cudaStream_t st) {
   if (R == 0) return MEDUSA_OK;
+  cudaError_t e;
   if (dtype == MEDUSA_F32)
-    topk_rows_kernel<float><<<R, kThreads, 0, st>>>((const float*)x, V, s, idx, val);
+    e = launch_pdl(topk_rows_kernel<float>, dim3(R), dim3(kThreads), 0, st, (const float*)x, V, s,
+                   idx, val);
   else
-    topk_rows_kernel<__nv_bfloat16><<<R, kThreads, 0, st>>>((const __nv_bfloat16*)x, V, s, idx,
-                                                            val);
-  cudaError_t e = cudaGetLastError();
+    e = launch_pdl(topk_rows_kernel<__nv_bfloat16>, dim3(R), dim3(kThreads), 0, st,
+                   (const __nv_bfloat16*)x, V, s, idx, val);
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "topk_rows_kernel launch");
 }
 
 int topk_keys_launch(const uint64_t* keys, int R, int C, int s, int32_t* idx, float* val,
                      cudaStream_t st) {
   if (R == 0) return MEDUSA_OK;
-  topk_keys_kernel<<<R, kThreads, 0, st>>>(keys, C, s, idx, val);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(topk_keys_kernel, dim3(R), dim3(kThreads), 0, st, keys, C, s, idx, val);
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "topk_keys_kernel launch");
 }
 

@@ -15,6 +15,9 @@ __global__ void build_tree_kernel(const int32_t* __restrict__ head_rank,
                                   const int32_t* __restrict__ topk,
                                   const int32_t* __restrict__ L, int B, int N, int Ks,
                                   int32_t* __restrict__ tok, int32_t* __restrict__ pos) {
+  // nothing in this kernel runs ahead of its predecessor
+  griddep_launch_dependents();
+  griddep_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= B * N) return;
   const int b = i / N, n = i - b * N;
@@ -29,9 +32,10 @@ int build_tree_launch(const medusa_tree* t, const int32_t* root, const int32_t* 
                       const int32_t* L, int B, int32_t* tok, int32_t* pos, cudaStream_t st) {
   const int total = B * t->N;
   if (total == 0) return MEDUSA_OK;
-  build_tree_kernel<<<(total + 255) / 256, 256, 0, st>>>(t->d_head_rank, t->d_depth, root, topk,
-                                                         L, B, t->N, t->K * t->s, tok, pos);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(build_tree_kernel, dim3((total + 255) / 256), dim3(256), 0, st,
+                             t->d_head_rank, t->d_depth, root, topk, L, B, t->N, t->K * t->s, tok,
+                             pos);
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "build_tree_kernel launch");
 }
 
