@@ -8,7 +8,10 @@
 //
 // Query rows of a (sequence, kv-head) are the tree nodes x the GQA group,
 // packed 128 to an MMA tile.  A CTA takes one 128-row query tile and one key
-// chunk of one (sequence, kv-head).  Per 128-key tile t:
+// chunk of one (sequence, kv-head); the grid's slowest index runs over the
+// sequences longest first (a permutation computed on the device), so the
+// long CTAs start first and the tail of the launch is made of short ones.
+// Per 128-key tile t:
 //   S  = Q K^T      tcgen05.mma (M 128, N 128, K 128): Q and K K-major in
 //                   smem (TMA, 128-byte swizzle), S into TMEM buffer t mod 3,
 //                   issued while the softmax of tile t-1 runs
@@ -156,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   griddep_wait();  // prefix lengths and the K/V cache may come from the kernel ahead
   const int qt = blockIdx.x, chunk = blockIdx.y, bk = blockIdx.z;
-  const int b = bk / p.Hkv, kvh = bk - b * p.Hkv;
+  const int rank = bk / p.Hkv, kvh = bk - rank * p.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* sQ = sm;
   uint8_t* sK = sm + TILE;
@@ -173,6 +176,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* mma_done = pv_done + 3;
   uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  int* seq_slot = (int*)(tmem_slot + 2);
+
+  // Sequence of this CTA: the one of rank `rank` by decreasing prefix length
+  // (ties: lower index first).  Every CTA ranks the B lengths itself (one
+  // thread per sequence); beyond kThreads sequences the order is the index.
+  int b = rank;
+  if (p.B > 1 && p.B <= kThreads) {
+    if ((int)threadIdx.x < p.B) {
+      const int i = threadIdx.x;
+      const int li = p.L[i];
+      int r = 0;
+      for (int j = 0; j < p.B; ++j) {
+        const int lj = p.L[j];
+        r += (lj > li || (lj == li && j < i)) ? 1 : 0;
+      }
+      if (r == rank) *seq_slot = i;
+    }
+    __syncthreads();
+    b = *seq_slot;
+  }
 
   const int Lb = p.L[b];
   const bool seq_ok = Lb >= 0 && (long long)Lb + p.N <= p.Lcap;
