@@ -76,6 +76,20 @@ const char* medusa_version(void);
  */
 int medusa_device_status(int* status, int clear);
 
+/*
+ * Failure-detection self-test; the pages have no counterpart (it checks the
+ * library's own bounded device waits).  Launches one CTA on `stream` (a
+ * cudaStream_t, NULL = default stream) whose single thread waits, with the
+ * same bounded wait every kernel of the library uses, for an mbarrier phase
+ * that nothing completes, giving up after `limit_ms` milliseconds of global
+ * time (1 <= limit_ms <= 2000).  The wait runs out, the kernel raises the
+ * device status word and returns normally: afterwards medusa_device_status()
+ * reports MEDUSA_ERR_TIMEOUT and the CUDA context stays usable.  Returns
+ * MEDUSA_ERR_INVALID_ARG for a limit out of range, MEDUSA_ERR_CUDA if the
+ * launch fails; asynchronous otherwise.
+ */
+int medusa_selftest_wait_timeout(int limit_ms, void* stream);
+
 /* ------------------------------------------------------------------------
  * Tree plan.  [MD] "ツリーアテンションによる並列検証": each of the K heads
  * proposes its top-s tokens; their Cartesian product is pruned to a tree.

@@ -59,6 +59,14 @@ def device_status(clear: bool = True) -> int:
     return st.value
 
 
+def selftest_wait_timeout(limit_ms: int, device=None) -> None:
+    """Launch the library's bounded-wait self-test on the current stream: one
+    thread waits for a barrier phase that nothing completes, gives up after
+    limit_ms, raises the device status word and returns."""
+    L.check(L.lib().medusa_selftest_wait_timeout(int(limit_ms), _stream(device)),
+            "medusa_selftest_wait_timeout")
+
+
 def tree_plan_host(K: int, s: int, N: int):
     """Host-only tree plan: (parent[N], depth[N], rank_path[N][K], anc_mask[N][W]) tensors."""
     W = (N + 31) // 32

@@ -130,22 +130,27 @@ __device__ __forceinline__ bool mbar_try_wait_for(uint64_t* bar, uint32_t parity
       : "memory");
   return ok != 0u;
 }
-// Bounded wait for phase `parity` of `bar`.  Returns false (and raises the
-// device status word and the CTA's abort flag) if it ran out, or if another
-// role of the CTA already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile int* abort_flag) {
+// Bounded wait for phase `parity` of `bar` (limit_ns of global time).
+// Returns false (and raises the device status word and the CTA's abort flag)
+// if it ran out, or if another role of the CTA already aborted.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity,
+                                                volatile int* abort_flag,
+                                                unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (;;) {
     if (mbar_try_wait_for(bar, parity, 200000u)) return true;
     if (abort_flag != nullptr && *abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       atomicOr(&g_dev_status, DEV_TIMEOUT);
       if (abort_flag != nullptr) *abort_flag = 1;
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          volatile int* abort_flag) {
+  return mbar_wait_limit(bar, parity, abort_flag, kWaitLimitNs);
 }
 
 // ---------------------------------------------------------------- TMA

@@ -210,7 +210,33 @@ bool dtype_ok(int dt) { return dt == MEDUSA_F32 || dt == MEDUSA_BF16; }
 
 using namespace medusa;
 
+namespace medusa {
+namespace selftest {
+// One thread waits for phase 0 of a barrier that no thread arrives at.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_limit(&bar, 0u, &abort_flag, limit_ns);
+}
+}  // namespace selftest
+}  // namespace medusa
+
 extern "C" {
+
+int medusa_selftest_wait_timeout(int limit_ms, void* stream) {
+  if (limit_ms < 1 || limit_ms > 2000)
+    return fail(MEDUSA_ERR_INVALID_ARG, "limit_ms must be in [1, 2000]");
+  selftest::selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(
+      (unsigned long long)limit_ms * 1000000ull);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "selftest_wait_kernel launch");
+}
 
 const char* medusa_last_error(void) { return t_last_error.c_str(); }
 
