@@ -18,7 +18,7 @@
 //   softmax         two warpgroups, one per 64-key half of the tile; a thread
 //                   owns one query row of one half: one TMEM read of its 64
 //                   scores, prefix limit / ancestor-bitmask mask, the row max
-//                   of the tile from both halves (exchanged through TMEM),
+//                   of the tile from both halves (exchanged through smem),
 //                   one running max per row with lazy rescaling (the
 //                   reference max moves only when it grows by more than 2^8;
 //                   the O row is then rescaled in TMEM once the previous P.V
@@ -50,7 +50,8 @@ constexpr uint32_t HALF = 128 * 64 * 2;  // 64-column half of a 128-row bf16 til
 constexpr uint32_t TILE = 2 * HALF;      // 32 KB
 constexpr int kStages = 3;
 constexpr size_t kDataBytes = (1 + 2 * kStages) * (size_t)TILE;  // Q | K ring | V ring
-constexpr size_t SMEM = 1024 + kDataBytes + 256;
+constexpr size_t kXchBytes = 2 * 2 * BM * sizeof(uint16_t);  // row-max exchange
+constexpr size_t SMEM = 1024 + kDataBytes + 256 + kXchBytes;
 constexpr float kRescale = 8.0f;  // log2 of the growth that forces a rescale
 static_assert(MEDUSA_MAX_N == 256, "ancestor words are selected for at most 4 x 64 nodes");
 
@@ -140,6 +141,13 @@ __device__ __forceinline__ void mask_half(float (&v)[64], int j, int hf, const R
   }
 }
 
+// bf16 bits of x rounded toward +inf (so the rounded value is >= x).
+__device__ __forceinline__ uint32_t bf16_bits_up(float x) {
+  uint32_t u = __float_as_uint(x);
+  if (!(u & 0x80000000u)) u += 0xFFFFu;  // non-negative: away from zero
+  return u >> 16;                          // negative: toward zero
+}
+
 __device__ __forceinline__ float max64(const float (&v)[64]) {
   float mx[8];
 #pragma unroll
@@ -177,6 +185,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   int* seq_slot = (int*)(tmem_slot + 2);
+  // [tile parity][key half][row]: each half's tile row max, bf16 rounded up
+  uint16_t* xch = (uint16_t*)(sm + kDataBytes + 256);
 
   // Sequence of this CTA: the one of rank `rank` by decreasing prefix length
   // (ties: lower index first).  Every CTA ranks the B lengths itself (one
@@ -363,13 +373,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       err = err || !__all_sync(0xffffffffu, good);
       float v[64];
       float tmax = -INFINITY;
+      // Both halves of a row use max(round_up(max_0), round_up(max_1)): the
+      // same value in both, and an upper bound of the row's tile max.  The
+      // parity double buffer is free again two barriers later.
+      uint16_t* xrow = xch + (size_t)(t & 1) * 2 * BM + r;
       if (!err && warp_live) {
         tc_fence_after();
         tmem_ld64(tS, v);
         mask_half(v, t, hf, rg, p.N, am);
-        tmax = max64(v) * p.qscale;  // scale > 0
-        tmem_st1(tS + 32u, tmax);   // column 32 of the half is not overwritten by P
-        tc_fence_before();
+        const uint32_t mine = bf16_bits_up(max64(v) * p.qscale);  // scale > 0
+        tmax = __uint_as_float(mine << 16);
+        xrow[hf * BM] = (uint16_t)mine;
       }
       if (bar_red_or(3 + q4, 64, err)) {
         ok = false;
@@ -382,8 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&p_full[bf]);
         continue;
       }
-      tc_fence_after();
-      tmax = fmaxf(tmax, tmem_ld1(tmem + lane_base + (uint32_t)(bf * 128 + (hf ^ 1) * 64 + 32)));
+      tmax = fmaxf(tmax, __uint_as_float((uint32_t)xrow[(hf ^ 1) * BM] << 16));
       const bool grow_m = tmax > m_used + kRescale;  // the same in both partners
       // warp-uniform branch: the TMEM accesses and the vote are collective
       if (__any_sync(0xffffffffu, grow_m)) {
@@ -422,9 +435,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         float x0, x1, e0, e1;
         f2_unpack(f2_fma(f2_pack(v[2 * c2], v[2 * c2 + 1]), q2, m2), x0, x1);
         if ((c2 & 3) == 3) {
+          // a masked key gives 2^-126 here rather than 0: negligible next
+          // to the row sum (>= 1 once a key is visible), and wiped by the
+          // zero rescale while the row has seen no visible key
           exp2_fma2(x0, x1, e0, e1);
-          e0 = (v[2 * c2] == -INFINITY) ? 0.f : e0;
-          e1 = (v[2 * c2 + 1] == -INFINITY) ? 0.f : e1;
         } else {
           e0 = ex2_approx(x0);
           e1 = ex2_approx(x1);
