@@ -234,7 +234,7 @@ class OracleSampler:
 def run_reference(args, cfg, world, rank):
     if rank != 0:
         return 0
-    t_setup = time.time()
+    t_setup = time.perf_counter()
     x = gen_inputs(cfg, "cpu", seed=0)
     from oracle import medusa_oracle as O
     plan = O.tree_plan(cfg.K, cfg.s, cfg.N)
