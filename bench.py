@@ -31,6 +31,7 @@ from medusa_head_speculative_02_b200.synthetic import CONFIGS, gen_inputs  # noq
 DEFAULT_CONFIG = "7b_b1"
 METRIC = "verify steps/s"
 EVENT_EVERY = 8  # timed steps per step whose heads / attention calls are bracketed by events
+DECODE_STEPS = 128  # chained steps of the decode-loop measurement
 
 
 # ---------------------------------------------------------------------------- helpers
@@ -339,6 +340,33 @@ def run_ours(args, cfg, world, rank, local):
     barrier()
     e2e = aggregate(Ke, e0.elapsed_time(e1) / 1000.0, world, dev)
 
+    # Multi-step decode: the next token of each step is the next root and its
+    # new lengths the next prefix lengths; one step is captured into a CUDA
+    # graph and DECODE_STEPS replays run back to back.  Every rank takes the
+    # same collective steps whether or not its capture worked.
+    dec_err, dec_s, dec_alen = None, 0.0, 0.0
+    loop = None
+    try:
+        from medusa_head_speculative_02_b200.decode import DecodeLoop
+        loop = DecodeLoop(cfg, dev, seed=rank, max_steps=DECODE_STEPS)
+        loop.capture()
+        torch.cuda.synchronize(dev)
+    except Exception as ex:  # reported in the JSON line, the main result stands
+        dec_err = f"{type(ex).__name__}: {ex}"[:300]
+    barrier()
+    if dec_err is None:
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for _ in range(DECODE_STEPS):
+            loop.step()
+        d1.record(stream)
+        torch.cuda.synchronize(dev)
+        dec_s = d0.elapsed_time(d1) / 1000.0
+        grown = (loop.st.x["prefix_len"].long() - loop._init["prefix_len"].long()).float()
+        dec_alen = (grown.mean().item() / DECODE_STEPS) - 1.0
+    dec = aggregate(DECODE_STEPS, dec_s if dec_err is None else 1.0, world, dev)
+    del loop
+
     peaks = measured_peaks()
     hb = st.heads_bytes()
     ab = st.attention_bytes()
@@ -379,6 +407,13 @@ def run_ours(args, cfg, world, rank, local):
                 "kernels": {"tree_attention": {"achieved": attn_gbs, "unit": "GB/s",
                                                "frac": attn_gbs / peaks["hbm_gbs"],
                                                "algorithmic_bytes": ab, "avg_ms": attn_ms}},
+                "decode_loop": ({"steps": DECODE_STEPS, "cuda_graph": True,
+                                 "steps_per_s": dec["value"],
+                                 "tokens_per_s": dec["value"] * cfg.B * (1.0 + dec_alen),
+                                 "mean_accept_len": dec_alen,
+                                 "note": "next token -> next root, new lengths -> next prefix "
+                                         "lengths; one captured step replayed per step"}
+                                if dec_err is None else {"error": dec_err}),
                 "e2e": {"value": e2e["value"], "unit": "steps/s",
                         "h2d_bytes_per_step": io.h2d_bytes(),
                         "d2h_bytes_per_step": io.d2h_bytes(), "steps": Ke},

@@ -41,10 +41,11 @@ class MedusaConfig:
     delta: float = 0.6
     plant_p: float = 0.4     # Geometric(p) planted accept length
     boost: float = 8.0
+    headroom: int = 0        # extra cache slots (room for the prefix to grow across steps)
 
     @property
     def Lcap(self) -> int:
-        return self.L_hi + self.N
+        return self.L_hi + self.N + self.headroom
 
     @property
     def torch_dtype(self):
