@@ -20,6 +20,9 @@ Sources (page title, then section):
        in one pass and the longest matching prefix is accepted.
   [FR] "Medusa" (glossaire) - "Attention en arbre": each node sees only its
        ancestors; the longest path whose tokens are all valid is accepted.
+  [ZH] "Medusa：基于多Token预测的LLM推理加速" - "3.3 贪婪vs采样验证": greedy
+       verification takes the argmax; sampling verification draws the token
+       from softmax(logits / temperature).
   Workload definition (tree scoring rule prod 0.5^r_i * 0.8^depth, sizes,
   tolerances) comes from the five workload configurations of this project.
 
@@ -29,7 +32,9 @@ by (depth asc, tuple lexicographic asc); the ancestor mask includes the node
 itself; kv-head of query head h is h // (Hq/Hkv); temperature divides the
 logits before both p and H; strict '>' in the typical test; the deepest
 accepted node wins, ties to the lowest node index; next token = argmax of
-the last accepted node's row; tree positions are prefix_len + depth.
+the last accepted node's row; tree positions are prefix_len + depth; the
+sampled next token is drawn from the last accepted node's row by Gumbel-max
+with SplitMix64 noise keyed by (seed, call offset, sequence, vocab index).
 
 Parity: every function here is pinned by tests/test_oracle_pins.py against
 closed forms, library routines or brute force (see each docstring).
@@ -45,7 +50,8 @@ __all__ = [
     "f64", "tree_score", "tree_plan", "silu", "heads_forward", "topk_row",
     "topk", "build_tree", "tree_attention", "row_argmax", "accept_greedy",
     "typical_row_stats", "typical_threshold", "accept_typical", "kv_compact",
-    "ancestors_or_self", "heads_hidden", "heads_logits",
+    "ancestors_or_self", "heads_hidden", "heads_logits", "splitmix64",
+    "uniform24", "gumbel32", "sample_next",
 ]
 
 
@@ -369,3 +375,73 @@ def kv_compact(k_cache, v_cache, prefix_len, accept_len, accept_nodes):
             v_new[b, L[b] + j] = v_old[b, L[b] + nodes[b, j]]
         new_len[b] = L[b] + 1 + A[b]
     return k_new, v_new, new_len
+
+
+# ---------------------------------------------------------------------------
+# Sampled next token.  [ZH] "3.3 贪婪vs采样验证": with temperature 0 the token
+# is the argmax, otherwise a draw from softmax(logits / temperature).
+# READING (the pages fix no generator): the draw is Gumbel-max, i.e. the
+# argmax of logits / T + G_v with G_v = -log(-log(U_v)) i.i.d. standard
+# Gumbel, which is distributed exactly as softmax(logits / T) (Gumbel 1954;
+# the "Gumbel-max trick"); U_v comes from the counter-based SplitMix64
+# generator (Steele, Lea & Flood, "Fast splittable pseudorandom number
+# generators", OOPSLA 2014) at counter index ((offset * B) + b) * V + v.
+# The decision is taken in fp32, the precision of the kernel.
+# ---------------------------------------------------------------------------
+_GAMMA = np.uint64(0x9E3779B97F4A7C15)
+
+
+def splitmix64(seed: int, idx) -> np.ndarray:
+    """Output number idx (0-based) of SplitMix64 started at state ``seed``:
+    the state after idx + 1 steps is seed + (idx + 1) * gamma (mod 2^64),
+    then the published finaliser (xor-shift 30, multiply, xor-shift 27,
+    multiply, xor-shift 31)."""
+    with np.errstate(over="ignore"):
+        x = np.uint64(seed) + (np.asarray(idx, dtype=np.uint64) + np.uint64(1)) * _GAMMA
+        z = (x ^ (x >> np.uint64(30))) * np.uint64(0xBF58476D1CE4E5B9)
+        z = (z ^ (z >> np.uint64(27))) * np.uint64(0x94D049BB133111EB)
+        return z ^ (z >> np.uint64(31))
+
+
+def uniform24(seed: int, idx) -> np.ndarray:
+    """fp32 uniforms in (0, 1): the top 24 bits of the SplitMix64 output plus
+    one half, times 2^-24 (exact in fp32, never 0 or 1)."""
+    top = (splitmix64(seed, idx) >> np.uint64(40)).astype(np.float32)
+    return ((top + np.float32(0.5)) * np.float32(2.0 ** -24)).astype(np.float32)
+
+
+def gumbel32(u: np.ndarray) -> np.ndarray:
+    """Standard Gumbel noise -log(-log(u)) in fp32."""
+    u = np.asarray(u, dtype=np.float32)
+    return (-np.log(-np.log(u))).astype(np.float32)
+
+
+def sample_next(vlogits, accept_len, accept_nodes, temperature: float, seed: int,
+                offset: int):
+    """Next token of every sequence drawn from the row of its last accepted
+    node n_a = accept_nodes[b][accept_len[b]].  temperature == 0: argmax
+    (lowest index on ties).  Otherwise argmax_v of z_v = fl(fl(l_v * (1/T)) +
+    G_v) in fp32 (ties: lowest index).  Returns (next_tok [B], gap [B]) where
+    gap is the fp32 distance between the best and second-best z (inf for the
+    argmax), so that a test can tell decisions too close to call."""
+    A = _i64(accept_len)
+    nodes = _i64(accept_nodes)
+    B = A.shape[0]
+    V = vlogits.shape[-1]
+    nxt = np.zeros(B, dtype=np.int64)
+    gap = np.full(B, np.inf)
+    inv_t = np.float32(1.0) / np.float32(temperature) if temperature > 0 else None
+    for b in range(B):
+        n_a = int(nodes[b, int(A[b])])
+        row = f64(vlogits[b, n_a]).astype(np.float32)   # exact: fp32 / bf16 inputs
+        if inv_t is None:
+            nxt[b] = int(np.argmax(row))
+            continue
+        idx = (np.uint64(offset) * np.uint64(B) + np.uint64(b)) * np.uint64(V) + \
+            np.arange(V, dtype=np.uint64)
+        z = (row * inv_t).astype(np.float32) + gumbel32(uniform24(seed, idx))
+        z = z.astype(np.float32)
+        nxt[b] = int(np.argmax(z))
+        srt = np.sort(z)
+        gap[b] = float(srt[-1]) - float(srt[-2])
+    return nxt, gap

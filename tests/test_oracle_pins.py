@@ -391,3 +391,77 @@ def test_kv_compact_equals_gather():
             idx[L[b] + j] = L[b] + nodes[b, j]
         np.testing.assert_array_equal(nk[b], kc[b].index_select(0, idx).numpy())
         np.testing.assert_array_equal(nv[b], vc[b].index_select(0, idx).numpy())
+
+
+# ----------------------------------------------------------------------------
+# Sampled next token (Gumbel-max over SplitMix64 noise)
+# ----------------------------------------------------------------------------
+def test_splitmix64_known_answers():
+    """The generator's first outputs from state 0 (tests/golden/splitmix64_seed0.txt)."""
+    rows = [ln.split() for ln in open(__import__("os").path.join(GOLDEN, "splitmix64_seed0.txt"))
+            if ln.strip() and not ln.startswith("#")]
+    idx = np.array([int(r[0]) for r in rows])
+    want = [int(r[1], 16) for r in rows]
+    assert [int(v) for v in O.splitmix64(0, idx)] == want
+
+
+def test_splitmix64_counter_form_equals_sequential_generator():
+    """Output i of the counter form = the (i+1)-th output of the stepping
+    generator (state += gamma, then the finaliser), for an arbitrary seed."""
+    M = (1 << 64) - 1
+    seed = 0x0123456789ABCDEF
+    x, seq = seed, []
+    for _ in range(12):
+        x = (x + 0x9E3779B97F4A7C15) & M
+        z = x
+        z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & M
+        z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & M
+        seq.append(z ^ (z >> 31))
+    assert [int(v) for v in O.splitmix64(seed, np.arange(12))] == seq
+
+
+def test_uniform24_range_and_uniformity():
+    u = O.uniform24(7, np.arange(200_000))
+    assert u.dtype == np.float32 and (u > 0).all() and (u < 1).all()
+    counts = np.bincount((u * 64).astype(np.int64), minlength=64)
+    exp = len(u) / 64
+    chi2 = float(((counts - exp) ** 2 / exp).sum())
+    assert chi2 < 110.0          # df = 63, p ~ 1e-4
+    # consecutive counters are uncorrelated
+    assert abs(np.corrcoef(u[:-1], u[1:])[0, 1]) < 0.01
+
+
+def test_gumbel_noise_moments():
+    """Standard Gumbel: mean = Euler-Mascheroni constant, variance pi^2 / 6."""
+    g = O.gumbel32(O.uniform24(11, np.arange(400_000))).astype(np.float64)
+    assert abs(g.mean() - 0.5772156649) < 0.01
+    assert abs(g.var() - math.pi ** 2 / 6) < 0.03
+
+
+def test_sample_next_frequencies_follow_softmax():
+    """Draws over many call offsets follow softmax(l / T) (chi-square)."""
+    l = np.array([2.0, 1.0, 0.5, 0.0, -1.0, 3.0], dtype=np.float32)
+    T = 0.8
+    vlog = torch.from_numpy(l).view(1, 1, 6)
+    A, nodes = np.array([0]), np.array([[0, -1]])
+    n = 20_000
+    hits = np.zeros(6)
+    for off in range(n):
+        t, _ = O.sample_next(vlog, A, nodes, T, seed=5, offset=off)
+        hits[t[0]] += 1
+    p = np.exp(l / T - (l / T).max())
+    p /= p.sum()
+    chi2 = float(((hits - n * p) ** 2 / (n * p)).sum())
+    assert chi2 < 20.5           # df = 5, p = 0.001
+
+
+def test_sample_next_temperature_zero_is_argmax_of_last_accepted_row():
+    g = torch.Generator().manual_seed(4)
+    vlog = torch.randn(3, 5, 50, generator=g)
+    A = np.array([0, 2, 1])
+    nodes = np.array([[0, -1, -1], [0, 3, 4], [0, 2, -1]])
+    t, _ = O.sample_next(vlog, A, nodes, 0.0, seed=1, offset=0)
+    assert list(t) == [int(vlog[0, 0].argmax()), int(vlog[1, 4].argmax()), int(vlog[2, 2].argmax())]
+    # a tiny temperature with a clear winner also picks the argmax
+    t2, _ = O.sample_next(vlog, A, nodes, 1e-3, seed=1, offset=3)
+    assert list(t2) == list(t)
