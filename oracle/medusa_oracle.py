@@ -51,7 +51,7 @@ __all__ = [
     "topk", "build_tree", "tree_attention", "row_argmax", "accept_greedy",
     "typical_row_stats", "typical_threshold", "accept_typical", "kv_compact",
     "ancestors_or_self", "heads_hidden", "heads_logits", "splitmix64",
-    "uniform24", "gumbel32", "sample_next",
+    "uniform01", "gumbel32", "sample_next",
 ]
 
 
@@ -385,7 +385,8 @@ def kv_compact(k_cache, v_cache, prefix_len, accept_len, accept_nodes):
 # Gumbel, which is distributed exactly as softmax(logits / T) (Gumbel 1954;
 # the "Gumbel-max trick"); U_v comes from the counter-based SplitMix64
 # generator (Steele, Lea & Flood, "Fast splittable pseudorandom number
-# generators", OOPSLA 2014) at counter index ((offset * B) + b) * V + v.
+# generators", OOPSLA 2014) at counter index ((offset * B) + b) * V + v,
+# as (top 23 bits + 1/2) * 2^-23.
 # The decision is taken in fp32, the precision of the kernel.
 # ---------------------------------------------------------------------------
 _GAMMA = np.uint64(0x9E3779B97F4A7C15)
@@ -403,11 +404,12 @@ def splitmix64(seed: int, idx) -> np.ndarray:
         return z ^ (z >> np.uint64(31))
 
 
-def uniform24(seed: int, idx) -> np.ndarray:
-    """fp32 uniforms in (0, 1): the top 24 bits of the SplitMix64 output plus
-    one half, times 2^-24 (exact in fp32, never 0 or 1)."""
-    top = (splitmix64(seed, idx) >> np.uint64(40)).astype(np.float32)
-    return ((top + np.float32(0.5)) * np.float32(2.0 ** -24)).astype(np.float32)
+def uniform01(seed: int, idx) -> np.ndarray:
+    """fp32 uniforms in (0, 1): the top 23 bits t of the SplitMix64 output,
+    (t + 1/2) * 2^-23.  Every step is exact in fp32 (t + 1/2 < 2^23 needs 24
+    significant bits), so u lies in [2^-24, 1 - 2^-24]: never 0 or 1."""
+    top = (splitmix64(seed, idx) >> np.uint64(41)).astype(np.float32)
+    return ((top + np.float32(0.5)) * np.float32(2.0 ** -23)).astype(np.float32)
 
 
 def gumbel32(u: np.ndarray) -> np.ndarray:
@@ -439,7 +441,7 @@ def sample_next(vlogits, accept_len, accept_nodes, temperature: float, seed: int
             continue
         idx = (np.uint64(offset) * np.uint64(B) + np.uint64(b)) * np.uint64(V) + \
             np.arange(V, dtype=np.uint64)
-        z = (row * inv_t).astype(np.float32) + gumbel32(uniform24(seed, idx))
+        z = (row * inv_t).astype(np.float32) + gumbel32(uniform01(seed, idx))
         z = z.astype(np.float32)
         nxt[b] = int(np.argmax(z))
         srt = np.sort(z)

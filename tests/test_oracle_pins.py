@@ -420,8 +420,22 @@ def test_splitmix64_counter_form_equals_sequential_generator():
     assert [int(v) for v in O.splitmix64(seed, np.arange(12))] == seq
 
 
-def test_uniform24_range_and_uniformity():
-    u = O.uniform24(7, np.arange(200_000))
+def test_uniform01_extremes_are_exact_and_inside_the_interval():
+    """The smallest and largest 23-bit values map exactly to 2^-24 and
+    1 - 2^-24 in fp32 (a construction that rounded the top value up to 1
+    would give infinite Gumbel noise)."""
+    top = np.array([0, 1, (1 << 23) - 2, (1 << 23) - 1], dtype=np.float32)
+    u = ((top + np.float32(0.5)) * np.float32(2.0 ** -23)).astype(np.float32)
+    assert u[0] == np.float32(2.0 ** -24) and u[-1] == np.float32(1 - 2.0 ** -24)
+    assert (u < 1).all() and (u > 0).all() and np.isfinite(O.gumbel32(u)).all()
+    # and the oracle's uniforms are exactly of that form
+    v = O.uniform01(3, np.arange(1000))
+    t = (O.splitmix64(3, np.arange(1000)) >> np.uint64(41)).astype(np.float64)
+    np.testing.assert_array_equal(v.astype(np.float64), (t + 0.5) * 2.0 ** -23)
+
+
+def test_uniform01_range_and_uniformity():
+    u = O.uniform01(7, np.arange(200_000))
     assert u.dtype == np.float32 and (u > 0).all() and (u < 1).all()
     counts = np.bincount((u * 64).astype(np.int64), minlength=64)
     exp = len(u) / 64
@@ -433,7 +447,7 @@ def test_uniform24_range_and_uniformity():
 
 def test_gumbel_noise_moments():
     """Standard Gumbel: mean = Euler-Mascheroni constant, variance pi^2 / 6."""
-    g = O.gumbel32(O.uniform24(11, np.arange(400_000))).astype(np.float64)
+    g = O.gumbel32(O.uniform01(11, np.arange(400_000))).astype(np.float64)
     assert abs(g.mean() - 0.5772156649) < 0.01
     assert abs(g.var() - math.pi ** 2 / 6) < 0.03
 
