@@ -12,6 +12,8 @@
  *        matching prefix).
  *   [FR] "Medusa" (glossaire), "Attention en arbre" (each node sees only its
  *        ancestors; the longest valid path is accepted).
+ *   [ZH] "Medusa：基于多Token预测的LLM推理加速", "3.3 贪婪vs采样验证" (greedy
+ *        versus sampling verification).
  *
  * Conventions shared by every call:
  *   - Return value: MEDUSA_OK (0) or a negative medusa_status.  On error
@@ -277,6 +279,28 @@ int medusa_kv_compact(void* k_cache, void* v_cache, const int32_t* prefix_len,
                       const int32_t* accept_len, const int32_t* accept_nodes,
                       int B, int Hkv, int dh, int Lcap, int K, int dtype,
                       int32_t* new_len, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Sampled next token.  [ZH] "3.3 贪婪vs采样验证": greedy verification takes
+ * the argmax, sampling verification draws from softmax(logits / T).  For
+ * every sequence b the token is drawn from the verify row
+ * vlogits[b][n_a][0..V) of its last accepted node n_a =
+ * accept_nodes[b][accept_len[b]] (accept_len / accept_nodes [B][K+1] as the
+ * accept calls write them; N = tree nodes).  temperature == 0: the argmax
+ * (lowest index on ties).  temperature > 0: argmax_v of
+ * fl(fl(l_v * (1/T)) + G_v) in fp32, G_v = -log(-log(U_v)) standard Gumbel
+ * noise (Gumbel-max: a draw from softmax(l / T)), U_v = (t + 1/2) * 2^-23
+ * with t the top 23 bits of output number ((offset * B) + b) * V + v of
+ * SplitMix64 started at `seed` (Steele, Lea & Flood, OOPSLA 2014).  The
+ * result depends only on (seed, offset) and the inputs: pass a new offset
+ * for every call that must draw fresh noise.  A sequence whose accept_len
+ * is outside [0, K] or whose node is outside [0, N) gets next_tok = -1.
+ * temperature must be finite and >= 0.  Writes next_tok [B] only.
+ * ------------------------------------------------------------------------ */
+int medusa_sample_next(const void* vlogits, int dtype, const int32_t* accept_len,
+                       const int32_t* accept_nodes, int B, int N, int V, int K,
+                       float temperature, uint64_t seed, uint64_t offset,
+                       int32_t* next_tok, void* stream);
 
 #ifdef __cplusplus
 }

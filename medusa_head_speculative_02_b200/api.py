@@ -244,6 +244,25 @@ def medusa_accept_typical(vlogits, tree_tok, tree: Tree, temperature: float, eps
     return alen, anodes, nxt
 
 
+def medusa_sample_next(vlogits, accept_len, accept_nodes, temperature: float, seed: int,
+                       offset: int, out=None):
+    """Next token of every sequence drawn from softmax(row / temperature) of its
+    last accepted node's verify row (Gumbel-max over counter-based noise;
+    temperature 0 = argmax)."""
+    B, N, V = vlogits.shape
+    _need(vlogits, "vlogits")
+    K = accept_nodes.shape[1] - 1
+    _need(accept_len, "accept_len", torch.int32, (B,))
+    _need(accept_nodes, "accept_nodes", torch.int32, (B, K + 1))
+    out = torch.empty(B, dtype=torch.int32, device=vlogits.device) if out is None else out
+    L.check(L.lib().medusa_sample_next(_ptr(vlogits), _dt(vlogits), _ptr(accept_len),
+                                       _ptr(accept_nodes), B, N, V, K, float(temperature),
+                                       int(seed) & ((1 << 64) - 1), int(offset) & ((1 << 64) - 1),
+                                       _ptr(out), _stream(vlogits.device)),
+            "medusa_sample_next")
+    return out
+
+
 def medusa_kv_compact(k_cache, v_cache, prefix_len, accept_len, accept_nodes, K: int,
                       new_len=None):
     B, Lcap, Hkv, dh = k_cache.shape
