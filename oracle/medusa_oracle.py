@@ -32,7 +32,9 @@ by (depth asc, tuple lexicographic asc); the ancestor mask includes the node
 itself; kv-head of query head h is h // (Hq/Hkv); temperature divides the
 logits before both p and H; strict '>' in the typical test; the deepest
 accepted node wins, ties to the lowest node index; next token = argmax of
-the last accepted node's row; tree positions are prefix_len + depth; the
+the last accepted node's row; tree positions are prefix_len + depth; with
+one temperature per head, the candidates of depth D are verified at the
+temperature of head D; the
 sampled next token is drawn from the last accepted node's row by Gumbel-max
 with SplitMix64 noise keyed by (seed, call offset, sequence, vocab index).
 
@@ -51,7 +53,7 @@ __all__ = [
     "topk", "build_tree", "tree_attention", "row_argmax", "accept_greedy",
     "typical_row_stats", "typical_threshold", "accept_typical", "kv_compact",
     "ancestors_or_self", "heads_hidden", "heads_logits", "splitmix64",
-    "uniform01", "gumbel32", "sample_next",
+    "uniform01", "gumbel32", "sample_next", "temperature_by_depth",
 ]
 
 
@@ -325,25 +327,42 @@ def typical_threshold(H: float, eps: float, delta: float) -> float:
     return min(eps, delta * np.exp(-H))
 
 
-def accept_typical(vlogits, tree_tok, plan: dict, temperature: float,
+def temperature_by_depth(temperature, K: int) -> list:
+    """T[D] for the candidates of depth D = 1..K (index 0 unused).  A scalar
+    applies to every depth.  READING of the per-head temperatures ([ZH]
+    "4.2 温度调优", one temperature per Medusa head): head D proposes the
+    nodes of depth D, and those are verified on their parent's row at T[D]."""
+    if np.ndim(temperature) == 0:
+        return [float(temperature)] * (K + 1)
+    t = [float(x) for x in temperature]
+    if len(t) != K:
+        raise ValueError("one temperature per head")
+    return [t[0]] + t
+
+
+def accept_typical(vlogits, tree_tok, plan: dict, temperature,
                    eps: float = 0.09, delta: float = 0.6):
     """Typical acceptance ([MD] "候補選択：Typical Acceptance").
 
     Node n != 0 is accepted iff its parent is accepted and
     p_parent(tok[n]) > min(eps, delta * exp(-H(p_parent))) with p = softmax of
-    the parent's verify row at ``temperature``.  Also returns, per (b, n), the
+    the parent's verify row at the temperature of n's depth (a scalar, or one
+    per head: ``temperature_by_depth``).  Also returns, per (b, n), the
     relative margin |p - thr| / thr of each node's own decision (used by the
     tests to flag decisions too close to call in any finite precision).
     """
     tok = _i64(tree_tok)
     B, N = tok.shape
     K = plan["K"]
+    T = temperature_by_depth(temperature, K)
     alen = np.zeros(B, dtype=np.int64)
     anodes = np.full((B, K + 1), -1, dtype=np.int64)
     nxt = np.zeros(B, dtype=np.int64)
     margin = np.full((B, N), np.inf)
     for b in range(B):
-        stats = [typical_row_stats(vlogits[b, n], temperature) for n in range(N)]
+        # every child of a row has the same depth: one temperature per row
+        stats = [typical_row_stats(vlogits[b, n], T[min(int(plan["depth"][n]) + 1, K)])
+                 for n in range(N)]
         acc = np.zeros(N, dtype=bool)
         acc[0] = True
         for n in range(1, N):

@@ -479,3 +479,39 @@ def test_sample_next_temperature_zero_is_argmax_of_last_accepted_row():
     # a tiny temperature with a clear winner also picks the argmax
     t2, _ = O.sample_next(vlog, A, nodes, 1e-3, seed=1, offset=3)
     assert list(t2) == list(t)
+
+
+# ----------------------------------------------------------------------------
+# Typical acceptance with one temperature per head
+# ----------------------------------------------------------------------------
+def test_typical_per_head_equal_temperatures_is_the_scalar_rule():
+    cfg = MedusaConfig("t", "f32", B=2, d=8, V=64, K=4, s=3, N=16, Hq=1, Hkv=1, dh=8,
+                       L_lo=4, L_hi=4, plant_p=0.2)
+    plan = O.tree_plan(cfg.K, cfg.s, cfg.N)
+    g = torch.Generator().manual_seed(8)
+    topk_idx = torch.stack([torch.randperm(cfg.V, generator=g)[:cfg.s * cfg.K].view(cfg.K, cfg.s)
+                            for _ in range(cfg.B)])
+    tok, _ = O.build_tree(plan, [1, 2], topk_idx, [4, 4])
+    vlog = plant_verify_logits(cfg, plan["parent"], tok, seed=8).double()
+    a = O.accept_typical(vlog, tok, plan, 0.7)
+    b = O.accept_typical(vlog, tok, plan, [0.7] * cfg.K)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_typical_per_head_temperature_decides_its_own_depth():
+    """Hand case: chain tree (s = 1), V = 8.  The root row favours token 0 by
+    3 nats; node 1 carries token 1.  At T = 0.1 its probability is ~e^-30
+    (rejected); at T = 10 the row is nearly uniform: H ~ ln 8, threshold
+    min(0.09, 0.6 / 8.0...) ~ 0.075 < p(1) = 1 / (7 + e^0.3) ~ 0.12 (accepted).
+    Node 2 (depth 2, token 2) sits on node 1's row, which is uniform: p = 1/8
+    > min(0.09, 0.6/8) = 0.075 at any temperature."""
+    plan = O.tree_plan(2, 1, 3)
+    assert [int(x) for x in plan["depth"]] == [0, 1, 2]
+    V = 8
+    vlog = np.zeros((1, 3, V))
+    vlog[0, 0, 0] = 3.0
+    tok = np.array([[5, 1, 2]])
+    for T, want in (([0.1, 1.0], 0), ([10.0, 1.0], 2), ([10.0, 0.05], 2)):
+        alen, nodes, _, _ = O.accept_typical(vlog, tok, plan, T)
+        assert int(alen[0]) == want, (T, alen)
