@@ -242,6 +242,22 @@ int medusa_accept_typical(const void* vlogits, int dtype,
                           size_t ws_bytes, void* stream);
 
 /*
+ * Typical acceptance with one temperature per head.  [ZH] "4.2 温度调优"
+ * tunes a temperature per Medusa head; reading: head D proposes the
+ * candidates of depth D, and each is verified on its parent's row at
+ * temperatures[D-1] (a host array of K floats, each finite and > 0; the
+ * workspace is medusa_accept_workspace_size's).  With all K equal this is
+ * medusa_accept_typical.  next_tok is the argmax of the last accepted row.
+ */
+int medusa_accept_typical_per_head(const void* vlogits, int dtype,
+                                   const int32_t* tree_tok,
+                                   const medusa_tree_t* tree, int B, int V,
+                                   const float* temperatures, float eps,
+                                   float delta, int32_t* accept_len,
+                                   int32_t* accept_nodes, int32_t* next_tok,
+                                   void* ws, size_t ws_bytes, void* stream);
+
+/*
  * medusa_accept_greedy without a workspace argument, for callers that cannot
  * allocate device memory: code that runs where cudaMalloc and allocating
  * libraries are off limits (for example a serving loop whose device memory

@@ -244,6 +244,28 @@ def medusa_accept_typical(vlogits, tree_tok, tree: Tree, temperature: float, eps
     return alen, anodes, nxt
 
 
+def medusa_accept_typical_per_head(vlogits, tree_tok, tree: Tree, temperatures, eps: float = 0.09,
+                                   delta: float = 0.6, out=None, ws=None):
+    """Typical acceptance with one temperature per head (the candidates of
+    depth D are verified at temperatures[D-1])."""
+    B, N, V = vlogits.shape
+    _need(vlogits, "vlogits")
+    _need(tree_tok, "tree_tok", torch.int32, (B, N))
+    temps = [float(t) for t in temperatures]
+    if len(temps) != tree.K:
+        raise ValueError(f"{len(temps)} temperatures for {tree.K} heads")
+    arr = (C.c_float * tree.K)(*temps)
+    alen, anodes, nxt = out if out is not None else _accept_outputs(B, tree.K, vlogits.device)
+    need = accept_workspace_size(tree, B, V)
+    if ws is None or ws.numel() < need:
+        ws = _ws(need, vlogits.device)
+    L.check(L.lib().medusa_accept_typical_per_head(
+        _ptr(vlogits), _dt(vlogits), _ptr(tree_tok), tree.handle, B, V, arr, float(eps),
+        float(delta), _ptr(alen), _ptr(anodes), _ptr(nxt), _ptr(ws), ws.numel(),
+        _stream(vlogits.device)), "medusa_accept_typical_per_head")
+    return alen, anodes, nxt
+
+
 def medusa_sample_next(vlogits, accept_len, accept_nodes, temperature: float, seed: int,
                        offset: int, out=None):
     """Next token of every sequence drawn from softmax(row / temperature) of its

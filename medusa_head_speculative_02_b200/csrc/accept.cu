@@ -34,6 +34,13 @@ constexpr int kRedThreads = 256;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Per-depth scale of typical acceptance: z[D] = log2(e) / T_D for the
+// candidates of depth D = 1..K (z[0] = z[1]); a row at depth d is reduced at
+// the scale of its children, z[min(d + 1, K)].
+struct ZTab {
+  float z[MEDUSA_MAX_K + 1];
+};
+
 struct RowPart {
   uint64_t key;
   float m, Z, S, pad;
@@ -128,12 +135,18 @@ __device__ __forceinline__ void red_consume(RedState& st, const float (&x)[NV], 
 
 template <typename T, bool TYPICAL>
 __global__ void __launch_bounds__(kRedThreads)
-    row_reduce_kernel(const T* __restrict__ vlog, int V, int chunk, int splits, float zscale,
+    row_reduce_kernel(const T* __restrict__ vlog, int V, int chunk, int splits, ZTab zt,
+                      const int32_t* __restrict__ depth, int N, int K,
                       RowPart* __restrict__ parts) {
   // nothing in this kernel runs ahead of its predecessor
   griddep_launch_dependents();
   griddep_wait();
   const size_t row = blockIdx.x;
+  float zscale = 0.f;
+  if (TYPICAL) {
+    const int dc = depth[row % (size_t)N] + 1;
+    zscale = zt.z[dc < K ? dc : K];
+  }
   const int sp = blockIdx.y;
   const int lo = sp * chunk;
   const int hi = min(V, lo + chunk);
@@ -210,7 +223,7 @@ __global__ void __launch_bounds__(MEDUSA_MAX_N)
     accept_walk_kernel(const T* __restrict__ vlog, const RowPart* __restrict__ parts, int splits,
                        const int32_t* __restrict__ tok, const int32_t* __restrict__ parent,
                        const int32_t* __restrict__ depth, const uint32_t* __restrict__ anc, int N,
-                       int W, int K, int V, float zscale, float eps, float delta,
+                       int W, int K, int V, ZTab zt, float eps, float delta,
                        int32_t* __restrict__ accept_len, int32_t* __restrict__ accept_nodes,
                        int32_t* __restrict__ next_tok) {
   // nothing in this kernel runs ahead of its predecessor
@@ -252,7 +265,8 @@ __global__ void __launch_bounds__(MEDUSA_MAX_N)
     if (TYPICAL) {
       if (t >= 0 && t < V) {
         const float x = to_f32(vlog[((size_t)b * N + par) * V + t]);
-        const float p = exp2f(x * zscale - mrow[par]) / zrow[par];
+        // the parent's row was reduced at the scale of n's depth
+        const float p = exp2f(x * zt.z[depth[n]] - mrow[par]) / zrow[par];
         c = p > thr[par];
       }
     } else {
@@ -334,7 +348,11 @@ int accept_launch(const AcceptArgs& a, cudaStream_t st) {
   const AccPlan P = make_plan(rows, a.V);
   if (a.ws_bytes < P.total) return fail(MEDUSA_ERR_INVALID_ARG, "workspace too small for accept");
   RowPart* parts = (RowPart*)a.ws;
-  const float zscale = a.typical ? kLog2e / a.temperature : 0.f;
+  ZTab zt;
+  for (int D = 0; D <= MEDUSA_MAX_K; ++D) {
+    const int i = D < 1 ? 0 : (D > a.tree->K ? a.tree->K - 1 : D - 1);
+    zt.z[D] = a.typical && a.tree->K > 0 ? kLog2e / a.temps[i < 0 ? 0 : i] : 0.f;
+  }
   dim3 g1(rows, P.splits);
   const int walk_threads = (N + 31) / 32 * 32;
   const medusa_tree* t = a.tree;
@@ -342,11 +360,11 @@ int accept_launch(const AcceptArgs& a, cudaStream_t st) {
 #define MEDUSA_ACC(T, TYP)                                                                     \
   do {                                                                                         \
     le = launch_pdl(row_reduce_kernel<T, TYP>, g1, dim3(kRedThreads), 0, st, (const T*)a.vlog, \
-                    a.V, P.chunk, P.splits, zscale, parts);                                    \
+                    a.V, P.chunk, P.splits, zt, t->d_depth, N, t->K, parts);                   \
     if (le == cudaSuccess)                                                                     \
       le = launch_pdl(accept_walk_kernel<T, TYP>, dim3(a.B), dim3(walk_threads), 0, st,        \
                       (const T*)a.vlog, parts, P.splits, a.tok, t->d_parent, t->d_depth,       \
-                      t->d_anc, N, t->W, t->K, a.V, zscale, a.eps, a.delta, a.accept_len,      \
+                      t->d_anc, N, t->W, t->K, a.V, zt, a.eps, a.delta, a.accept_len,          \
                       a.accept_nodes, a.next_tok);                                             \
   } while (0)
   if (a.dtype == MEDUSA_F32) {
@@ -418,16 +436,17 @@ int accept_greedy_noalloc_launch(const void* vlog, int dtype, const int32_t* tok
   if (rc) return rc;
   dim3 g1((unsigned)rows, P.splits);
   const int walk_threads = (N + 31) / 32 * 32;
+  const ZTab zt0 = {};  // greedy: no scale
   cudaError_t le = cudaSuccess;
 #define MEDUSA_ACC_STATIC(T)                                                                     \
   do {                                                                                           \
     le = launch_pdl(row_reduce_kernel<T, false>, g1, dim3(kRedThreads), 0, st, (const T*)vlog, V, \
-                    P.chunk, P.splits, 0.f, parts);                                              \
+                    P.chunk, P.splits, zt0, t->d_depth, N, t->K, parts);                         \
     if (le == cudaSuccess)                                                                       \
       le = launch_pdl(accept_walk_kernel<T, false>, dim3(B), dim3(walk_threads), 0, st,          \
                       (const T*)vlog,                                                            \
                       parts, P.splits, tok, t->d_parent, t->d_depth, t->d_anc, N, t->W, t->K, V, \
-                      0.f, 0.f, 0.f, accept_len, accept_nodes, next_tok);                        \
+                      zt0, 0.f, 0.f, accept_len, accept_nodes, next_tok);                        \
   } while (0)
   if (dtype == MEDUSA_F32)
     MEDUSA_ACC_STATIC(float);

@@ -127,7 +127,8 @@ struct AcceptArgs {
   const medusa_tree* tree;
   int B, V;
   bool typical;
-  float temperature, eps, delta;
+  float temps[MEDUSA_MAX_K];  // typical: temperature of the candidates of depth 1..K
+  float eps, delta;
   int32_t* accept_len;
   int32_t* accept_nodes;
   int32_t* next_tok;

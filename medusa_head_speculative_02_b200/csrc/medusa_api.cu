@@ -443,23 +443,47 @@ size_t medusa_accept_workspace_size(const medusa_tree_t* tree, int B, int V) {
   return accept_workspace(tree, B, V);
 }
 
+// temps: host array of the per-depth temperatures (K entries) or NULL for
+// the single temperature T.
 static int accept_common(const void* vlogits, int dtype, const int32_t* tree_tok,
                          const medusa_tree_t* tree, int B, int V, bool typical, float T,
-                         float eps, float delta, int32_t* accept_len, int32_t* accept_nodes,
-                         int32_t* next_tok, void* ws, size_t ws_bytes, void* stream) {
+                         const float* temps, float eps, float delta, int32_t* accept_len,
+                         int32_t* accept_nodes, int32_t* next_tok, void* ws, size_t ws_bytes,
+                         void* stream) {
   int rc = check_tree(tree);
   if (rc) return rc;
   if (!dtype_ok(dtype)) return fail(MEDUSA_ERR_INVALID_ARG, "bad dtype");
   if (B < 0 || V < 1) return fail(MEDUSA_ERR_INVALID_ARG, "bad shape");
-  if (typical && !(T > 0.f && std::isfinite(T) && std::isfinite(eps) && std::isfinite(delta)))
-    return fail(MEDUSA_ERR_INVALID_ARG, "typical acceptance needs T > 0 and finite eps, delta");
+  float tk[MEDUSA_MAX_K];
+  for (int i = 0; i < MEDUSA_MAX_K; ++i) tk[i] = (temps && i < tree->K) ? temps[i] : T;
+  if (typical) {
+    bool good = std::isfinite(eps) && std::isfinite(delta);
+    for (int i = 0; i < tree->K; ++i) good = good && tk[i] > 0.f && std::isfinite(tk[i]);
+    if (!good)
+      return fail(MEDUSA_ERR_INVALID_ARG,
+                  "typical acceptance needs temperatures > 0 and finite eps, delta");
+  }
   if (B == 0) return MEDUSA_OK;
   if (!vlogits || !tree_tok || !accept_len || !accept_nodes || !next_tok)
     return fail(MEDUSA_ERR_INVALID_ARG, "NULL pointer");
   const size_t need = accept_workspace(tree, B, V);
   if (!ws || ws_bytes < need) return fail(MEDUSA_ERR_INVALID_ARG, "workspace too small");
-  AcceptArgs a{vlogits, dtype, tree_tok, tree, B, V, typical, T, eps, delta,
-               accept_len, accept_nodes, next_tok, ws, ws_bytes};
+  AcceptArgs a{};
+  a.vlog = vlogits;
+  a.dtype = dtype;
+  a.tok = tree_tok;
+  a.tree = tree;
+  a.B = B;
+  a.V = V;
+  a.typical = typical;
+  for (int i = 0; i < MEDUSA_MAX_K; ++i) a.temps[i] = tk[i];
+  a.eps = eps;
+  a.delta = delta;
+  a.accept_len = accept_len;
+  a.accept_nodes = accept_nodes;
+  a.next_tok = next_tok;
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
   return accept_launch(a, (cudaStream_t)stream);
 }
 
@@ -467,16 +491,26 @@ int medusa_accept_greedy(const void* vlogits, int dtype, const int32_t* tree_tok
                          const medusa_tree_t* tree, int B, int V, int32_t* accept_len,
                          int32_t* accept_nodes, int32_t* next_tok, void* ws, size_t ws_bytes,
                          void* stream) {
-  return accept_common(vlogits, dtype, tree_tok, tree, B, V, false, 1.f, 0.f, 0.f, accept_len,
-                       accept_nodes, next_tok, ws, ws_bytes, stream);
+  return accept_common(vlogits, dtype, tree_tok, tree, B, V, false, 1.f, nullptr, 0.f, 0.f,
+                       accept_len, accept_nodes, next_tok, ws, ws_bytes, stream);
 }
 
 int medusa_accept_typical(const void* vlogits, int dtype, const int32_t* tree_tok,
                           const medusa_tree_t* tree, int B, int V, float temperature, float eps,
                           float delta, int32_t* accept_len, int32_t* accept_nodes,
                           int32_t* next_tok, void* ws, size_t ws_bytes, void* stream) {
-  return accept_common(vlogits, dtype, tree_tok, tree, B, V, true, temperature, eps, delta,
-                       accept_len, accept_nodes, next_tok, ws, ws_bytes, stream);
+  return accept_common(vlogits, dtype, tree_tok, tree, B, V, true, temperature, nullptr, eps,
+                       delta, accept_len, accept_nodes, next_tok, ws, ws_bytes, stream);
+}
+
+int medusa_accept_typical_per_head(const void* vlogits, int dtype, const int32_t* tree_tok,
+                                   const medusa_tree_t* tree, int B, int V,
+                                   const float* temperatures, float eps, float delta,
+                                   int32_t* accept_len, int32_t* accept_nodes, int32_t* next_tok,
+                                   void* ws, size_t ws_bytes, void* stream) {
+  if (!temperatures) return fail(MEDUSA_ERR_INVALID_ARG, "temperatures is NULL");
+  return accept_common(vlogits, dtype, tree_tok, tree, B, V, true, 1.f, temperatures, eps,
+                       delta, accept_len, accept_nodes, next_tok, ws, ws_bytes, stream);
 }
 
 int medusa_accept_greedy_noalloc(const void* vlogits, int dtype, const int32_t* tree_tok,

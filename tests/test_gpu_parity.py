@@ -235,6 +235,24 @@ def test_accept_typical(dtype, B, K, s, N, V, sigma, T):
     _check_typical(alen.cpu().numpy(), anodes.cpu().numpy(), nxt.cpu().numpy(), ref, plan, B)
 
 
+@pytest.mark.parametrize("dtype,B,K,s,N,V,temps", [
+    (torch.bfloat16, 4, 5, 10, 64, 32000, (0.5, 0.7, 1.0, 1.2, 1.5)),
+    (torch.float32, 3, 4, 3, 16, 1000, (2.0, 0.3, 1.0, 0.6)),
+    (torch.bfloat16, 2, 3, 4, 40, 5000, (0.7, 0.7, 0.7)),
+])
+def test_accept_typical_per_head(dtype, B, K, s, N, V, temps):
+    """One temperature per head: node of depth D verified at temps[D-1]."""
+    cfg = _small_cfg(dtype=dtype, B=B, K=K, s=s, N=N, V=V, sigma=1.0)
+    plan, tok, vlog = _accept_inputs(cfg, seed=B * 7 + N)
+    t = api.Tree(K, s, N)
+    alen, anodes, nxt = api.medusa_accept_typical_per_head(vlog, tok, t, temps, 0.09, 0.6)
+    ref = O.accept_typical(vlog, tok, plan, list(temps), 0.09, 0.6)
+    _check_typical(alen.cpu().numpy(), anodes.cpu().numpy(), nxt.cpu().numpy(), ref, plan, B)
+    if len(set(temps)) == 1:   # equal temperatures: the scalar entry point
+        a2, n2, x2 = api.medusa_accept_typical(vlog, tok, t, temps[0], 0.09, 0.6)
+        assert torch.equal(a2, alen) and torch.equal(n2, anodes) and torch.equal(x2, nxt)
+
+
 def test_accept_typical_uniform_rows_accept_lowest_deepest():
     """Uniform verify rows over V = 8: p = 1/8 exceeds min(0.09, 0.6/8) = 0.075,
     so every node is accepted and the deepest node with the lowest index wins."""
