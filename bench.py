@@ -32,6 +32,7 @@ DEFAULT_CONFIG = "7b_b1"
 METRIC = "verify steps/s"
 EVENT_EVERY = 8  # timed steps per step whose heads / attention calls are bracketed by events
 DECODE_STEPS = 128  # chained steps of the decode-loop measurement
+SAMPLE_REPS = 50    # timed calls of the sampled-next-token measurement
 
 
 # ---------------------------------------------------------------------------- helpers
@@ -340,6 +341,23 @@ def run_ours(args, cfg, world, rank, local):
     barrier()
     e2e = aggregate(Ke, e0.elapsed_time(e1) / 1000.0, world, dev)
 
+    # Sampled next token on this step's verify rows and accepted paths (one
+    # row of V logits per sequence), CUDA events around SAMPLE_REPS calls.
+    from medusa_head_speculative_02_b200 import api as _api
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    tok_buf = torch.empty(cfg.B, dtype=torch.int32, device=dev)
+    for i in range(3):
+        _api.medusa_sample_next(st.vlogits, st.accept_len, st.accept_nodes, 0.7, rank, i,
+                                out=tok_buf)
+    torch.cuda.synchronize(dev)
+    s0.record(stream)
+    for i in range(SAMPLE_REPS):
+        _api.medusa_sample_next(st.vlogits, st.accept_len, st.accept_nodes, 0.7, rank, 3 + i,
+                                out=tok_buf)
+    s1.record(stream)
+    torch.cuda.synchronize(dev)
+    sample_ms = s0.elapsed_time(s1) / SAMPLE_REPS
+
     # Multi-step decode: the next token of each step is the next root and its
     # new lengths the next prefix lengths; one step is captured into a CUDA
     # graph and DECODE_STEPS replays run back to back.  Every rank takes the
@@ -368,6 +386,7 @@ def run_ours(args, cfg, world, rank, local):
     del loop
 
     peaks = measured_peaks()
+    sample_bytes = cfg.B * cfg.V * (4 if cfg.dtype == "f32" else 2)
     hb = st.heads_bytes()
     ab = st.attention_bytes()
     heads_gbs = hb / (heads_ms / 1000.0) / 1e9
@@ -406,7 +425,13 @@ def run_ours(args, cfg, world, rank, local):
                              "algorithmic_bytes": hb, "avg_ms": heads_ms},
                 "kernels": {"tree_attention": {"achieved": attn_gbs, "unit": "GB/s",
                                                "frac": attn_gbs / peaks["hbm_gbs"],
-                                               "algorithmic_bytes": ab, "avg_ms": attn_ms}},
+                                               "algorithmic_bytes": ab, "avg_ms": attn_ms},
+                            "sample_next": {"avg_ms": sample_ms, "temperature": 0.7,
+                                            "algorithmic_bytes": sample_bytes,
+                                            "achieved": sample_bytes / (sample_ms / 1e3) / 1e9,
+                                            "unit": "GB/s",
+                                            "note": "one verify row per sequence; "
+                                                    "latency-bound at small batch"}},
                 "decode_loop": ({"steps": DECODE_STEPS, "cuda_graph": True,
                                  "steps_per_s": dec["value"],
                                  "tokens_per_s": dec["value"] * cfg.B * (1.0 + dec_alen),

@@ -307,16 +307,19 @@ int medusa_kv_compact(void* k_cache, void* v_cache, const int32_t* prefix_len,
  * fl(fl(l_v * (1/T)) + G_v) in fp32, G_v = -log(-log(U_v)) standard Gumbel
  * noise (Gumbel-max: a draw from softmax(l / T)), U_v = (t + 1/2) * 2^-23
  * with t the top 23 bits of output number ((offset * B) + b) * V + v of
- * SplitMix64 started at `seed` (Steele, Lea & Flood, OOPSLA 2014).  The
- * result depends only on (seed, offset) and the inputs: pass a new offset
- * for every call that must draw fresh noise.  A sequence whose accept_len
+ * SplitMix64 started at `seed` (Steele, Lea & Flood, OOPSLA 2014); offset =
+ * `offset` + *offset_dev when offset_dev (a device uint64, read when the
+ * kernel runs) is not NULL.  The result depends only on (seed, offset) and
+ * the inputs: pass a new offset for every call that must draw fresh noise
+ * (offset_dev lets a captured CUDA graph advance it on the device between
+ * replays).  A sequence whose accept_len
  * is outside [0, K] or whose node is outside [0, N) gets next_tok = -1.
  * temperature must be finite and >= 0.  Writes next_tok [B] only.
  * ------------------------------------------------------------------------ */
 int medusa_sample_next(const void* vlogits, int dtype, const int32_t* accept_len,
                        const int32_t* accept_nodes, int B, int N, int V, int K,
                        float temperature, uint64_t seed, uint64_t offset,
-                       int32_t* next_tok, void* stream);
+                       const uint64_t* offset_dev, int32_t* next_tok, void* stream);
 
 #ifdef __cplusplus
 }

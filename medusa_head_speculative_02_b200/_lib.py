@@ -24,7 +24,7 @@ SIGNATURES = {
     "medusa_device_status": (ci, [C.POINTER(ci), ci]),
     "medusa_selftest_wait_timeout": (ci, [ci, vp]),
     "medusa_sample_next": (ci, [vp, ci, vp, vp, ci, ci, ci, ci, C.c_float, C.c_uint64,
-                                C.c_uint64, vp, vp]),
+                                C.c_uint64, vp, vp, vp]),
     "medusa_tree_plan_host": (ci, [ci, ci, ci, vp, vp, vp, vp]),
     "medusa_tree_create": (ci, [ci, ci, ci, C.POINTER(vp)]),
     "medusa_tree_destroy": (ci, [vp]),

@@ -267,10 +267,11 @@ def medusa_accept_typical_per_head(vlogits, tree_tok, tree: Tree, temperatures, 
 
 
 def medusa_sample_next(vlogits, accept_len, accept_nodes, temperature: float, seed: int,
-                       offset: int, out=None):
+                       offset: int, out=None, offset_dev=None):
     """Next token of every sequence drawn from softmax(row / temperature) of its
     last accepted node's verify row (Gumbel-max over counter-based noise;
-    temperature 0 = argmax)."""
+    temperature 0 = argmax).  offset_dev: optional one-element int64 device
+    tensor added to ``offset`` when the kernel runs."""
     B, N, V = vlogits.shape
     _need(vlogits, "vlogits")
     K = accept_nodes.shape[1] - 1
@@ -280,7 +281,7 @@ def medusa_sample_next(vlogits, accept_len, accept_nodes, temperature: float, se
     L.check(L.lib().medusa_sample_next(_ptr(vlogits), _dt(vlogits), _ptr(accept_len),
                                        _ptr(accept_nodes), B, N, V, K, float(temperature),
                                        int(seed) & ((1 << 64) - 1), int(offset) & ((1 << 64) - 1),
-                                       _ptr(out), _stream(vlogits.device)),
+                                       _ptr(offset_dev), _ptr(out), _stream(vlogits.device)),
             "medusa_sample_next")
     return out
 

@@ -151,7 +151,8 @@ int kv_compact_launch(void* k, void* v, const int32_t* L, const int32_t* alen,
 // sampled next token (csrc/sample.cu)
 int sample_next_launch(const void* vlog, int dtype, const int32_t* alen, const int32_t* anodes,
                        int B, int N, int V, int K, float temperature, uint64_t seed,
-                       uint64_t offset, int32_t* next_tok, cudaStream_t st);
+                       uint64_t offset, const uint64_t* offset_dev, int32_t* next_tok,
+                       cudaStream_t st);
 
 int make_tmap_bf16(void* map /* CUtensorMap* */, const void* base, int rank,
                    const uint64_t* dims, const uint64_t* strides_bytes,

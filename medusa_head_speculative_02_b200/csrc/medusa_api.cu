@@ -544,8 +544,8 @@ int medusa_kv_compact(void* k_cache, void* v_cache, const int32_t* prefix_len,
 
 int medusa_sample_next(const void* vlogits, int dtype, const int32_t* accept_len,
                        const int32_t* accept_nodes, int B, int N, int V, int K,
-                       float temperature, uint64_t seed, uint64_t offset, int32_t* next_tok,
-                       void* stream) {
+                       float temperature, uint64_t seed, uint64_t offset,
+                       const uint64_t* offset_dev, int32_t* next_tok, void* stream) {
   if (!dtype_ok(dtype)) return fail(MEDUSA_ERR_INVALID_ARG, "bad dtype");
   if (B < 0 || N <= 0 || N > MEDUSA_MAX_N || V <= 0 || K < 0 || K > MEDUSA_MAX_K)
     return fail(MEDUSA_ERR_INVALID_ARG, "bad shape");
@@ -555,7 +555,7 @@ int medusa_sample_next(const void* vlogits, int dtype, const int32_t* accept_len
   if (!vlogits || !accept_len || !accept_nodes || !next_tok)
     return fail(MEDUSA_ERR_INVALID_ARG, "NULL pointer");
   return sample_next_launch(vlogits, dtype, accept_len, accept_nodes, B, N, V, K, temperature,
-                            seed, offset, next_tok, (cudaStream_t)stream);
+                            seed, offset, offset_dev, next_tok, (cudaStream_t)stream);
 }
 
 }  // extern "C"

@@ -105,3 +105,56 @@ def test_headroom_bounds_the_step_count():
     loop.step()
     with pytest.raises(RuntimeError):
         loop.step()
+
+
+CFG_TYP = CFG.scaled(name="decode_small_typical", accept="typical", temperature=0.8)
+
+
+def test_sampling_chain_graph_equals_eager_and_draws_fresh_noise():
+    steps = 4
+    loop = DecodeLoop(CFG_TYP, "cuda", seed=5, max_steps=steps + 1, sample_temperature=0.9,
+                      sample_seed=77)
+    eager = []
+    for _ in range(steps):
+        loop.step()
+        eager.append(_outputs(loop.st))
+    assert int(loop.draws.item()) == steps
+    loop.reset()
+    loop.capture()
+    for i in range(steps):
+        loop.step()
+        got = _outputs(loop.st)
+        for k, v in eager[i].items():
+            assert torch.equal(got[k], v), (i, k)
+    assert int(loop.draws.item()) == steps
+
+
+def test_sampling_chain_matches_oracle_chain():
+    """Typical acceptance, then the next token drawn at offset = step index."""
+    steps, T_s, seed_s = 3, 0.9, 123
+    loop = DecodeLoop(CFG_TYP, "cuda", seed=6, max_steps=steps, sample_temperature=T_s,
+                      sample_seed=seed_s)
+    st, cfg = loop.st, loop.cfg
+    plan = O.tree_plan(cfg.K, cfg.s, cfg.N)
+    vlog = st.vlogits.cpu()
+    L = st.x["prefix_len"].cpu().numpy().astype(np.int64)
+    root = st.x["root_tok"].cpu().numpy().astype(np.int64)
+    kc, vc = O.f64(st.x["k_cache"].cpu()), O.f64(st.x["v_cache"].cpu())
+    for step in range(steps):
+        loop.step()
+        torch.cuda.synchronize()
+        idx = st.topk_idx.cpu().numpy()
+        tok, _ = O.build_tree(plan, root, idx, L)
+        assert (st.tree_tok.cpu().numpy() == tok).all()
+        alen, anodes, _, margin = O.accept_typical(vlog, tok, plan, cfg.temperature, cfg.eps,
+                                                   cfg.delta)
+        assert (margin > 1e-5).all()          # no decision too close to call
+        assert (st.accept_len.cpu().numpy() == alen).all()
+        assert (st.accept_nodes.cpu().numpy() == anodes).all()
+        nxt, gap = O.sample_next(vlog, alen, anodes, T_s, seed_s, step)
+        got = st.next_tok.cpu().numpy()
+        assert ((got == nxt) | (gap < 1e-5)).all() and (gap >= 1e-5).all()
+        kc, vc, new_len = O.kv_compact(kc, vc, L, alen, anodes)
+        assert (st.new_len.cpu().numpy() == new_len).all()
+        assert np.array_equal(O.f64(st.x["k_cache"].cpu()), kc)
+        L, root = new_len, nxt

@@ -69,3 +69,13 @@ def test_sample_next_invalid_path_gives_minus_one():
     nodes[2, int(alen[2])] = 99   # node outside [0, N)
     got = api.medusa_sample_next(vlog.cuda(), alen.cuda(), nodes.cuda(), 0.5, 1, 1).cpu()
     assert got[1] == -1 and got[2] == -1 and got[0] >= 0
+
+
+def test_device_offset_adds_to_the_host_offset():
+    vlog, alen, nodes = _inputs(4, 16, 3000, 4, torch.bfloat16, 6)
+    v, a, n = vlog.cuda(), alen.cuda(), nodes.cuda()
+    dev_off = torch.tensor([5], dtype=torch.int64, device="cuda")
+    for host in (0, 3):
+        want = api.medusa_sample_next(v, a, n, 0.8, 9, host + 5)
+        got = api.medusa_sample_next(v, a, n, 0.8, 9, host, offset_dev=dev_off)
+        assert torch.equal(got, want)
