@@ -39,7 +39,8 @@ AttnPlan make_plan(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lca
   P.rblocks = (P.R + RB - 1) / RB;
   const long long base = (long long)P.rblocks * B * Hkv;
   const int sms = num_sms();
-  long long want = (4LL * sms + base - 1) / base;  // >= ~4 CTAs per SM in total
+  // >= ~4 CTAs per SM in total (an empty batch has nothing to split)
+  long long want = base > 0 ? (4LL * sms + base - 1) / base : 1;
   const int max_p = (Lcap + 255) / 256;           // >= 256 keys per chunk
   if (want < 1) want = 1;
   if (want > max_p) want = max_p;

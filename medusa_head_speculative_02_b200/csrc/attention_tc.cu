@@ -511,6 +511,7 @@ int attention_tc_chunks(int B, int Hq, int Hkv, int N, int Lcap) {
   const int G = Hq / Hkv;
   const long long R = (long long)N * G;
   const long long units = (long long)B * Hkv * ((R + BM - 1) / BM);
+  if (units <= 0) return 1;  // empty batch: nothing to split
   const int sms = num_sms();
   long long P = (2LL * sms + units - 1) / units;
   const long long max_p = ((long long)(Lcap - N) + 4 * BN - 1) / (4 * BN);  // >= 4 tiles each
