@@ -159,17 +159,24 @@ __global__ void __launch_bounds__(kRedThreads)
     const int nv = (hi - lo) / VEC;
     // a thread whose values are all -inf reports its first column
     if ((int)threadIdx.x < nv) st.bi = lo + (int)threadIdx.x * VEC;
-    // two 16-byte loads in flight per thread
-    for (int i = threadIdx.x; i < nv; i += 2 * kRedThreads) {
-      const bool two = i + kRedThreads < nv;
-      const uint4 w0 = __ldcs(p + i);
-      const uint4 w1 = two ? __ldcs(p + i + kRedThreads) : make_uint4(0u, 0u, 0u, 0u);
-      float x[VEC];
-      Lanes<T>::get(w0, x);
-      red_consume<TYPICAL, VEC>(st, x, lo + i * VEC, zscale);
-      if (two) {
-        Lanes<T>::get(w1, x);
-        red_consume<TYPICAL, VEC>(st, x, lo + (i + kRedThreads) * VEC, zscale);
+    // four 16-byte loads in flight per thread (enough bytes in flight per SM
+    // to cover the memory latency), folded in index order
+    constexpr int kUnroll = 4;
+    for (int i = threadIdx.x; i < nv; i += kUnroll * kRedThreads) {
+      uint4 w[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int iu = i + u * kRedThreads;
+        w[u] = iu < nv ? __ldcs(p + iu) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int iu = i + u * kRedThreads;
+        if (iu < nv) {
+          float x[VEC];
+          Lanes<T>::get(w[u], x);
+          red_consume<TYPICAL, VEC>(st, x, lo + iu * VEC, zscale);
+        }
       }
     }
   } else {
