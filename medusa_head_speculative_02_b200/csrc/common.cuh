@@ -285,33 +285,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
-// Warp-collective: 128 consecutive fp32 columns of this warp's 32 TMEM lanes
-// in one load instruction, plus its completion wait.
-__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float (&v)[128]) {
-  uint32_t r[128];
-#define MEDUSA_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), \
-                     "=r"(r[i + 4]), "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x128.b32 {"
-      "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
-      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
-      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,"
-      "%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
-      "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,"
-      "%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,"
-      "%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127"
-      "}, [%128];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : MEDUSA_R8(0), MEDUSA_R8(8), MEDUSA_R8(16), MEDUSA_R8(24), MEDUSA_R8(32), MEDUSA_R8(40),
-        MEDUSA_R8(48), MEDUSA_R8(56), MEDUSA_R8(64), MEDUSA_R8(72), MEDUSA_R8(80),
-        MEDUSA_R8(88), MEDUSA_R8(96), MEDUSA_R8(104), MEDUSA_R8(112), MEDUSA_R8(120)
-      : "r"(taddr)
-      : "memory");
-#undef MEDUSA_R8
-#pragma unroll
-  for (int i = 0; i < 128; ++i) v[i] = __uint_as_float(r[i]);
-}
 // Warp-collective: 64 consecutive fp32 columns, one load plus its wait.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
   uint32_t r[64];
@@ -391,34 +364,6 @@ __device__ __forceinline__ bool bar_red_or(int id, int n, bool pred) {
       : "memory");
   return r != 0;
 }
-// 2^x on the FMA/ALU pipes (offloads the MUFU unit): Cody-Waite split
-// x = n + f with n = round(x), obtained by adding 1.5 * 2^23, and
-// f in [-0.5, 0.5]; 2^f by the degree-3 polynomial that minimises the
-// maximum relative error on [-0.5, 0.5] (coefficients fitted by Remez
-// exchange: max relative error 7.5e-5, 1.5e-4 once evaluated in fp32);
-// 2^n by adding n to the exponent field.  For x <= 127; x < -126 returns
-// 2^-126 (callers zero masked entries themselves).
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const int n = __float_as_int(t) - 0x4B400000;
-  const float f = x - (t - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(0.05517166853f, f, 0.24261112511f), f, 0.69326096773f), f,
-                       0.99992805719f);
-  return __int_as_float(__float_as_int(p) + (n << 23));
-}
-// Non-blocking test of phase `parity` of `bar`.
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0u;
-}
 // Packed fp32 pairs (Blackwell f32x2 FMA / ADD): a 64-bit register holds
 // (lo, hi).
 __device__ __forceinline__ unsigned long long f2_pack(float lo, float hi) {
@@ -440,27 +385,31 @@ __device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsig
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
-// Two 2^x on the FMA pipe in packed form (same method as exp2_fma).
+// 2^x on the FMA/ALU pipes (offloads the MUFU unit), two lanes at a time
+// in packed fp32x2 arithmetic: Cody-Waite split x = n + f with n = round(x),
+// obtained by adding 1.5 * 2^23, and f in [-0.5, 0.5]; 2^f by the degree-3
+// polynomial that minimises the maximum relative error on [-0.5, 0.5]
+// (coefficients fitted by Remez exchange: max relative error 7.5e-5,
+// 1.5e-4 once evaluated in fp32); 2^n by adding n to the exponent field.
+// For x <= 127; x < -126 gives 2^-126.
+constexpr float kExp2C0 = 0.99992805719f;
+constexpr float kExp2C1 = 0.69326096773f;
+constexpr float kExp2C2 = 0.24261112511f;
+constexpr float kExp2C3 = 0.05517166853f;
 __device__ __forceinline__ void exp2_fma2(float x0, float x1, float& e0, float& e1) {
   const unsigned long long x2 = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
   const unsigned long long t2 = f2_add(x2, f2_pack(12582912.0f, 12582912.0f));
   const unsigned long long f2 = f2_add(x2, f2_add(t2, f2_pack(-12582912.0f, -12582912.0f)) ^
                                                0x8000000080000000ull);
   const unsigned long long p2 =
-      f2_fma(f2_fma(f2_fma(f2_pack(0.05517166853f, 0.05517166853f), f2,
-                           f2_pack(0.24261112511f, 0.24261112511f)),
-                    f2, f2_pack(0.69326096773f, 0.69326096773f)),
-             f2, f2_pack(0.99992805719f, 0.99992805719f));
+      f2_fma(f2_fma(f2_fma(f2_pack(kExp2C3, kExp2C3), f2, f2_pack(kExp2C2, kExp2C2)), f2,
+                    f2_pack(kExp2C1, kExp2C1)),
+             f2, f2_pack(kExp2C0, kExp2C0));
   float t0, t1, p0, p1;
   f2_unpack(t2, t0, t1);
   f2_unpack(p2, p0, p1);
   e0 = __int_as_float(__float_as_int(p0) + ((__float_as_int(t0) - 0x4B400000) << 23));
   e1 = __int_as_float(__float_as_int(p1) + ((__float_as_int(t1) - 0x4B400000) << 23));
-}
-// Two non-negative floats to a bf16x2 word (first argument in the low half),
-// rounding half up, with integer ops only (no conversion-pipe instruction).
-__device__ __forceinline__ uint32_t pack_bf16x2_pos(float lo, float hi) {
-  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
 }
 // Hardware base-2 exponential (MUFU ex2, approximate, flush-to-zero); used
 // where a few ulp are far below the bf16 rounding that follows.
