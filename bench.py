@@ -33,6 +33,7 @@ METRIC = "verify steps/s"
 EVENT_EVERY = 8  # timed steps per step whose heads / attention calls are bracketed by events
 DECODE_STEPS = 128  # chained steps of the decode-loop measurement
 SAMPLE_REPS = 50    # timed calls of the sampled-next-token measurement
+E2E_GRAPH_STEPS = 8  # end-to-end steps per captured CUDA graph
 
 
 # ---------------------------------------------------------------------------- helpers
@@ -277,7 +278,7 @@ def run_reference(args, cfg, world, rank):
 
 
 def run_ours(args, cfg, world, rank, local):
-    from medusa_head_speculative_02_b200.step import HostIO, VerifyStep
+    from medusa_head_speculative_02_b200.step import PipelinedHostIO, VerifyStep
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     st = VerifyStep(cfg, dev, seed=rank)
@@ -325,17 +326,21 @@ def run_ours(args, cfg, world, rank, local):
     ms_per_step = agg["seconds"] * 1000.0 / K
     alen = st.accept_len.float().mean().item()
 
-    # end to end through the public API with host buffers
-    io = HostIO(st)
-    Ke = max(10, K // 8)
-    for _ in range(3):
-        io.step()
+    # end to end through the public API with host buffers: every step copies
+    # its inputs from pinned host memory (the next step's on a copy stream,
+    # overlapped with this step's kernels; the tree K/V slots on the compute
+    # stream) and reads its results back
+    io = PipelinedHostIO(st)
+    io.capture(E2E_GRAPH_STEPS)     # E2E_GRAPH_STEPS steps per graph launch
+    Ke = E2E_GRAPH_STEPS * max(2, K // (8 * E2E_GRAPH_STEPS))
+    for _ in range(2):
+        io.replay()
     torch.cuda.synchronize(dev)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(Ke):
-        io.step()
+    for _ in range(Ke // E2E_GRAPH_STEPS):
+        io.replay()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -441,7 +446,13 @@ def run_ours(args, cfg, world, rank, local):
                                 if dec_err is None else {"error": dec_err}),
                 "e2e": {"value": e2e["value"], "unit": "steps/s",
                         "h2d_bytes_per_step": io.h2d_bytes(),
-                        "d2h_bytes_per_step": io.d2h_bytes(), "steps": Ke},
+                        "d2h_bytes_per_step": io.d2h_bytes(), "steps": Ke,
+                        "copies": "pinned host -> device every step; the next step's "
+                                  "hidden state, queries, verify logits, roots and lengths "
+                                  "on a copy stream overlapping this step, the tree K/V "
+                                  "slots on the compute stream",
+                        "launch": f"API calls and copies of {E2E_GRAPH_STEPS} steps captured "
+                                  f"once into a CUDA graph, replayed"},
                 "gpu_launches": st.launches_per_step() * K,
                 "clocks": clk}
     # CPU baseline: the oracle on rank 0 at N = 1 only

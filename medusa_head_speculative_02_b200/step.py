@@ -167,3 +167,117 @@ class HostIO:
         self.o_next.copy_(st.next_tok, non_blocking=True)
         self.o_len.copy_(st.new_len, non_blocking=True)
         self.o_topk.copy_(st.topk_idx, non_blocking=True)
+
+
+class PipelinedHostIO(HostIO):
+    """HostIO with the host->device copies of the next step overlapped with
+    the current step's kernels, and with few copies per step.
+
+    The per-step inputs that do not live in the KV cache (hidden state, tree
+    queries, verify logits, root tokens, prefix lengths) are packed into one
+    pinned host buffer and copied with one copy into one of two device
+    buffers, whose views the step reads: a copy stream fills the buffer of
+    step k+1 while step k runs on the compute stream, once the step that last
+    used that buffer has finished.  The tree K/V slots are written on the
+    compute stream at the start of each step (the previous step's attention
+    and compaction use the same cache).  The step writes its results into
+    views of one device buffer, read back with one copy.
+    """
+
+    _KEYS = ("h", "q", "root_tok", "prefix_len")
+
+    @staticmethod
+    def _pack(specs, align=256):
+        offs, total = [], 0
+        for _, t in specs:
+            total = (total + align - 1) // align * align
+            offs.append(total)
+            total += t.numel() * t.element_size()
+        return offs, total
+
+    def __init__(self, st: VerifyStep):
+        super().__init__(st)
+        c, dev = st.cfg, st.dev
+        ins = [("h", self.h), ("q", self.q), ("vlog", self.vlog), ("root_tok", self.root),
+               ("prefix_len", self.plen)]
+        offs, total = self._pack(ins)
+        self.host_in = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+        self.dev_in = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(2)]
+
+        def view(buf, off, t):
+            n = t.numel() * t.element_size()
+            return buf[off:off + n].view(t.dtype).view(t.shape)
+
+        for (name, t), off in zip(ins, offs):
+            view(self.host_in, off, t).copy_(t)
+        self.sets = [{name: view(buf, off, t) for (name, t), off in zip(ins, offs)}
+                     for buf in self.dev_in]
+        # results: views of one int32 device buffer, read back with one copy
+        outs = [("accept_len", self.o_alen), ("accept_nodes", self.o_nodes),
+                ("next_tok", self.o_next), ("new_len", self.o_len), ("topk_idx", self.o_topk)]
+        n_out = sum(t.numel() for _, t in outs)
+        self.dev_out = torch.empty(n_out, dtype=torch.int32, device=dev)
+        self.host_out = torch.empty(n_out, dtype=torch.int32, pin_memory=True)
+        o = 0
+        for name, t in outs:
+            setattr(st, name, self.dev_out[o:o + t.numel()].view(t.shape))
+            setattr(self, {"accept_len": "o_alen", "accept_nodes": "o_nodes", "next_tok": "o_next",
+                           "new_len": "o_len", "topk_idx": "o_topk"}[name],
+                    self.host_out[o:o + t.numel()].view(t.shape))
+            o += t.numel()
+        self.copy_stream = torch.cuda.Stream(dev)
+        self.ready = [torch.cuda.Event(), torch.cuda.Event()]
+        self.free = [torch.cuda.Event(), torch.cuda.Event()]
+
+    def h2d_bytes(self) -> int:
+        return self.host_in.numel() + sum(t.numel() * t.element_size()
+                                          for t in (self.tree_k, self.tree_v))
+
+    def _copy_inputs(self, j: int, wait_free: bool) -> None:
+        with torch.cuda.stream(self.copy_stream):
+            if wait_free:   # the step that used buffer j earlier in this run has finished
+                self.copy_stream.wait_event(self.free[j])
+            self.dev_in[j].copy_(self.host_in, non_blocking=True)
+            self.ready[j].record(self.copy_stream)
+
+    def run(self, n: int) -> None:
+        """n steps; the inputs of step k+1 are copied while step k computes.
+        Every event a run waits on is recorded within the same run, so a run
+        can also be captured into a CUDA graph (``capture``)."""
+        st, c = self.st, self.st.cfg
+        cs = torch.cuda.current_stream(st.dev)
+        if n <= 0:
+            return
+        self.copy_stream.wait_stream(cs)   # no copy starts before the work already queued
+        self._copy_inputs(0, wait_free=False)
+        for k in range(n):
+            j = k & 1
+            if k + 1 < n:
+                self._copy_inputs(j ^ 1, wait_free=k >= 1)
+            cs.wait_event(self.ready[j])
+            cur = self.sets[j]
+            for key in self._KEYS:
+                st.x[key] = cur[key]
+            st.vlogits = cur["vlog"]
+            for b in range(c.B):
+                st.x["k_cache"][b, self.L[b]:self.L[b] + c.N].copy_(self.tree_k[b], non_blocking=True)
+                st.x["v_cache"][b, self.L[b]:self.L[b] + c.N].copy_(self.tree_v[b], non_blocking=True)
+            st.run()
+            self.free[j].record(cs)
+            self.host_out.copy_(self.dev_out, non_blocking=True)
+
+    def capture(self, steps_per_graph: int = 8) -> None:
+        """Capture ``steps_per_graph`` pipelined steps (host copies included:
+        the graph's copy nodes read the pinned host buffers at every replay)
+        into a CUDA graph; ``replay()`` then runs them with one launch."""
+        dev = self.st.dev
+        self.run(2)   # library set-up (first-call attributes, tensor maps) outside the capture
+        torch.cuda.synchronize(dev)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.run(steps_per_graph)
+        torch.cuda.synchronize(dev)
+        self.steps_per_graph = steps_per_graph
+
+    def replay(self) -> None:
+        self.graph.replay()
