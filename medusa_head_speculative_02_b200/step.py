@@ -16,9 +16,9 @@ from . import api
 from .synthetic import MedusaConfig, gen_inputs, plant_verify_logits
 
 # kernels this library launches per call
-# (stage-1 GEMM, SiLU epilogue, stage-2 GEMM, top-s merge; attention on the
-# tensor-core path is a sequence-order kernel plus the attention kernel, and
-# a combine kernel follows when it splits the keys into chunks)
+# (heads: stage-1 GEMM, SiLU epilogue, stage-2 GEMM, top-s merge; attention:
+# the attention kernel, plus a combine kernel when it splits the keys into
+# chunks)
 LAUNCHES = {"heads": 4, "build_tree": 1, "tree_attention": 1, "accept": 2, "kv_compact": 1}
 
 
@@ -101,10 +101,8 @@ class VerifyStep:
         c = self.cfg
         n_acc = 2 if c.accept == "both" else 1
         chunks = api.attention_chunks(self.tree, c.B, c.Hq, c.Hkv, c.dh, c.Lcap, c.torch_dtype)
-        tc = c.dtype == "bf16" and c.dh == 128 and (128 % (c.Hq // c.Hkv)) == 0
         return (LAUNCHES["heads"] + LAUNCHES["build_tree"] + LAUNCHES["tree_attention"] +
-                (1 if tc else 0) + (1 if chunks > 1 else 0) + n_acc * LAUNCHES["accept"] +
-                LAUNCHES["kv_compact"])
+                (1 if chunks > 1 else 0) + n_acc * LAUNCHES["accept"] + LAUNCHES["kv_compact"])
 
     # algorithmic bytes --------------------------------------------------------
     def heads_bytes(self) -> int:
