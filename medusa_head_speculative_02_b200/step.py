@@ -176,10 +176,10 @@ class PipelinedHostIO(HostIO):
     pinned host buffer and copied with one copy into one of two device
     buffers, whose views the step reads: a copy stream fills the buffer of
     step k+1 while step k runs on the compute stream, once the step that last
-    used that buffer has finished.  The tree K/V slots are written on the
-    compute stream at the start of each step (the previous step's attention
-    and compaction use the same cache).  The step writes its results into
-    views of one device buffer, read back with one copy.
+    used that buffer has finished.  The tree K/V slots of step k go through
+    the copy stream too, ahead of that, as soon as step k-1 (whose attention
+    and compaction use the same cache) has finished.  The step writes its
+    results into views of one device buffer, read back with one copy.
     """
 
     _KEYS = ("h", "q", "root_tok", "prefix_len")
@@ -226,6 +226,7 @@ class PipelinedHostIO(HostIO):
         self.copy_stream = torch.cuda.Stream(dev)
         self.ready = [torch.cuda.Event(), torch.cuda.Event()]
         self.free = [torch.cuda.Event(), torch.cuda.Event()]
+        self.kv_ready = torch.cuda.Event()
 
     def h2d_bytes(self) -> int:
         return self.host_in.numel() + sum(t.numel() * t.element_size()
@@ -240,8 +241,12 @@ class PipelinedHostIO(HostIO):
 
     def run(self, n: int) -> None:
         """n steps; the inputs of step k+1 are copied while step k computes.
-        Every event a run waits on is recorded within the same run, so a run
-        can also be captured into a CUDA graph (``capture``)."""
+        All host->device copies go through the copy stream, in the order they
+        are needed: once step k-1 has finished, the tree K/V slots of step k
+        (which step k-1's attention and compaction used), then the packed
+        inputs of step k+1, which overlap step k's kernels.  Every event a
+        run waits on is recorded within the same run, so a run can also be
+        captured into a CUDA graph (``capture``)."""
         st, c = self.st, self.st.cfg
         cs = torch.cuda.current_stream(st.dev)
         if n <= 0:
@@ -250,16 +255,23 @@ class PipelinedHostIO(HostIO):
         self._copy_inputs(0, wait_free=False)
         for k in range(n):
             j = k & 1
+            with torch.cuda.stream(self.copy_stream):
+                if k >= 1:   # step k-1 has released the cache slots
+                    self.copy_stream.wait_event(self.free[j ^ 1])
+                for b in range(c.B):
+                    st.x["k_cache"][b, self.L[b]:self.L[b] + c.N].copy_(self.tree_k[b],
+                                                                        non_blocking=True)
+                    st.x["v_cache"][b, self.L[b]:self.L[b] + c.N].copy_(self.tree_v[b],
+                                                                        non_blocking=True)
+                self.kv_ready.record(self.copy_stream)
             if k + 1 < n:
                 self._copy_inputs(j ^ 1, wait_free=k >= 1)
             cs.wait_event(self.ready[j])
+            cs.wait_event(self.kv_ready)
             cur = self.sets[j]
             for key in self._KEYS:
                 st.x[key] = cur[key]
             st.vlogits = cur["vlog"]
-            for b in range(c.B):
-                st.x["k_cache"][b, self.L[b]:self.L[b] + c.N].copy_(self.tree_k[b], non_blocking=True)
-                st.x["v_cache"][b, self.L[b]:self.L[b] + c.N].copy_(self.tree_v[b], non_blocking=True)
             st.run()
             self.free[j].record(cs)
             self.host_out.copy_(self.dev_out, non_blocking=True)
