@@ -542,15 +542,10 @@ int attention_tc_run(const AttnArgs& a, int P, float* po, float2* pml, cudaStrea
     rc = make_tmap_bf16(&mV, a.v, 3, dims, strides, box);
     if (rc) return rc;
   }
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(tree_attn_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tree_attn_tc_kernel)");
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_done[64];
+  int rc = ensure_max_smem(tree_attn_tc_kernel, (int)SMEM, attr_done,
+                           "cudaFuncSetAttribute(tree_attn_tc_kernel)");
+  if (rc) return rc;
   TcAttnParams p;
   p.L = a.L;
   p.anc = t->d_anc;

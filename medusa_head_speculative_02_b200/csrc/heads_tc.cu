@@ -414,15 +414,10 @@ template <int NC>
 int launch_stage(const CUtensorMap& A, const CUtensorMap& Bm, const TcParams& p,
                  cudaStream_t st) {
   using C = TcCfg<NC>;
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(heads_tc_kernel<NC>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(heads_tc_kernel)");
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_done[64];  // one per instantiation of NC
+  int rc = ensure_max_smem(heads_tc_kernel<NC>, (int)C::SMEM, attr_done,
+                           "cudaFuncSetAttribute(heads_tc_kernel)");
+  if (rc) return rc;
   const int grid = p.units < num_sms() ? p.units : num_sms();
   cudaError_t e = launch_pdl(heads_tc_kernel<NC>, dim3(grid), dim3(kThreads), C::SMEM, st, A, Bm, p);
   if (e == cudaSuccess) e = cudaGetLastError();

@@ -5,6 +5,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <string>
 #include <vector>
 
@@ -29,6 +30,23 @@ namespace medusa {
 int fail(int code, const std::string& msg);
 int cuda_fail(cudaError_t e, const char* what);
 int num_sms();
+
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` once per device;
+// `done` is the call site's own per-device flag array (safe to call from
+// several host threads).
+template <typename K>
+int ensure_max_smem(K* kernel, int bytes, std::atomic<bool> (&done)[64], const char* what) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(MEDUSA_ERR_UNSUPPORTED, "device ordinal >= 64");
+  if (!done[dev].load(std::memory_order_acquire)) {
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    done[dev].store(true, std::memory_order_release);
+  }
+  return MEDUSA_OK;
+}
 
 // Launches a kernel of this library with programmatic stream serialization:
 // it may be scheduled before the kernel ahead of it in the stream has

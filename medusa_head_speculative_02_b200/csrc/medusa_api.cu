@@ -55,17 +55,17 @@ int cuda_fail(cudaError_t e, const char* what) {
 }
 
 int num_sms() {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
   if (dev >= 0 && dev < 64) {
-    if (!cache[dev]) {
-      int n = 0;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n <= 0) {
       if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
         n = 148;
-      cache[dev] = n;
+      cache[dev].store(n, std::memory_order_relaxed);
     }
-    return cache[dev];
+    return n;
   }
   return 148;
 }
