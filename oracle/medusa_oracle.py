@@ -53,7 +53,7 @@ __all__ = [
     "topk", "build_tree", "tree_attention", "row_argmax", "accept_greedy",
     "typical_row_stats", "typical_threshold", "accept_typical", "kv_compact",
     "ancestors_or_self", "heads_hidden", "heads_logits", "splitmix64",
-    "uniform01", "gumbel32", "sample_next", "temperature_by_depth",
+    "uniform01", "gumbel32", "sample_next", "temperature_by_depth", "topk_merge",
 ]
 
 
@@ -213,6 +213,24 @@ def topk(logits, s: int) -> np.ndarray:
 # r_D of head D (head D predicts D+1 steps ahead; the root carries the token
 # just produced by the base model).  READING: tree_pos = prefix_len + depth.
 # ---------------------------------------------------------------------------
+def topk_merge(vals, idxs, s: int):
+    """Top-s of candidate lists: vals, idxs [G][R][c] (index < 0 = empty
+    slot); per row r, the s best of all G * c candidates by value descending,
+    ties to the lower index.  Returns (idx [R][s], val [R][s]) with -1 / NaN
+    where fewer than s candidates exist."""
+    v = f64(vals)
+    ix = _i64(idxs)
+    G, R, c = ix.shape
+    out_i = np.full((R, s), -1, dtype=np.int64)
+    out_v = np.full((R, s), np.nan)
+    for r in range(R):
+        cand = [(v[g, r, j], ix[g, r, j]) for g in range(G) for j in range(c) if ix[g, r, j] >= 0]
+        cand.sort(key=lambda t: (-t[0], t[1]))
+        for j, (val, i) in enumerate(cand[:s]):
+            out_i[r, j], out_v[r, j] = i, val
+    return out_i, out_v
+
+
 def build_tree(plan: dict, root_tok, topk_idx, prefix_len):
     root = _i64(root_tok)
     tk = _i64(topk_idx)

@@ -515,3 +515,37 @@ def test_typical_per_head_temperature_decides_its_own_depth():
     for T, want in (([0.1, 1.0], 0), ([10.0, 1.0], 2), ([10.0, 0.05], 2)):
         alen, nodes, _, _ = O.accept_typical(vlog, tok, plan, T)
         assert int(alen[0]) == want, (T, alen)
+
+
+# ----------------------------------------------------------------------------
+# Merging per-shard top-s lists (vocabulary split across ranks)
+# ----------------------------------------------------------------------------
+def test_topk_merge_of_shard_lists_is_the_global_topk():
+    """Each shard's own top-s, with global indices, merged = top-s of the
+    whole row (brute force), for uneven shard sizes and ties."""
+    g = torch.Generator().manual_seed(12)
+    R, V, s = 7, 1000, 6
+    logits = torch.randn(R, V, generator=g, dtype=torch.float64)
+    logits[2, 100:110] = 5.0                       # a 10-way tie across shards
+    bounds = [0, 137, 500, 501, 1000]              # 4 shards, one of a single column
+    vals, idxs = [], []
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        k = min(s, b - a)
+        loc = O.topk(logits[:, a:b].numpy(), k)
+        v = np.take_along_axis(logits[:, a:b].numpy(), loc, axis=1)
+        vi = np.full((R, s), -1)
+        vv = np.zeros((R, s))
+        vi[:, :k], vv[:, :k] = loc + a, v
+        vals.append(vv)
+        idxs.append(vi)
+    mi, mv = O.topk_merge(np.stack(vals), np.stack(idxs), s)
+    want = O.topk(logits.numpy(), s)
+    np.testing.assert_array_equal(mi, want)
+    np.testing.assert_array_equal(mv, np.take_along_axis(logits.numpy(), want, axis=1))
+
+
+def test_topk_merge_pads_when_candidates_run_out():
+    vals = np.array([[[3.0, 1.0]], [[2.0, 0.0]]])
+    idxs = np.array([[[4, -1]], [[9, -1]]])
+    mi, mv = O.topk_merge(vals, idxs, 3)
+    assert mi.tolist() == [[4, 9, -1]] and mv[0, 0] == 3.0 and np.isnan(mv[0, 2])
