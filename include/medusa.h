@@ -297,6 +297,25 @@ int medusa_kv_compact(void* k_cache, void* v_cache, const int32_t* prefix_len,
                       int32_t* new_len, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Merge of top-s candidate lists from G vocabulary shards (heads whose W2
+ * rows are split across ranks: each rank's medusa_heads_forward top-s over
+ * its slice, gathered, then merged).  [MD] "ツリーアテンションによる並列検証":
+ * each head contributes its s most likely tokens.  Shard g's list for row
+ * r is val[g * shard_stride + r * c + j] fp32 and idx[...] int32 with the
+ * same offsets, j < c (index < 0: empty slot); shard_stride >= R * c
+ * elements (R * c for dense [G][R][c] arrays; 2 * R * c for the [G][2][R][c]
+ * buffer an all-gather of [values; ids] planes produces).  Shard g's indices
+ * are offset by v0[g] (device int32 [G]; NULL = no offset).  Per row r
+ * writes the s best candidates by value descending, ties to the lower
+ * (offset) index: out_idx [R][s] and, if non-NULL, out_val [R][s]; -1 / NaN
+ * where fewer than s candidates exist.  1 <= s <= MEDUSA_MAX_S.
+ * ------------------------------------------------------------------------ */
+int medusa_topk_merge(const float* val, const int32_t* idx,
+                      long long shard_stride, const int32_t* v0, int G, int R,
+                      int c, int s, int32_t* out_idx, float* out_val,
+                      void* stream);
+
+/* ------------------------------------------------------------------------
  * Sampled next token.  [ZH] "3.3 贪婪vs采样验证": greedy verification takes
  * the argmax, sampling verification draws from softmax(logits / T).  For
  * every sequence b the token is drawn from the verify row

@@ -23,6 +23,7 @@ SIGNATURES = {
     "medusa_version": (C.c_char_p, []),
     "medusa_device_status": (ci, [C.POINTER(ci), ci]),
     "medusa_selftest_wait_timeout": (ci, [ci, vp]),
+    "medusa_topk_merge": (ci, [vp, vp, C.c_longlong, vp, ci, ci, ci, ci, vp, vp, vp]),
     "medusa_sample_next": (ci, [vp, ci, vp, vp, ci, ci, ci, ci, C.c_float, C.c_uint64,
                                 C.c_uint64, vp, vp, vp]),
     "medusa_tree_plan_host": (ci, [ci, ci, ci, vp, vp, vp, vp]),

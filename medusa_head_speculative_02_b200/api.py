@@ -155,6 +155,37 @@ def medusa_topk(logits, s: int):
     return idx, val
 
 
+def _merge(val_ptr, idx_ptr, gs, G, R, c, s, v0, out, dev):
+    if v0 is not None:
+        _need(v0, "v0", torch.int32, (G,))
+    oi, ov = out if out is not None else (
+        torch.empty(R, s, dtype=torch.int32, device=dev),
+        torch.empty(R, s, dtype=torch.float32, device=dev))
+    L.check(L.lib().medusa_topk_merge(val_ptr, idx_ptr, gs, _ptr(v0), G, R, c, s, _ptr(oi),
+                                      _ptr(ov), _stream(dev)), "medusa_topk_merge")
+    return oi, ov
+
+
+def medusa_topk_merge(vals, idxs, s: int, v0=None, out=None):
+    """Top-s of G candidate lists per row: vals float32 / idxs int32
+    [G][R][c] (index < 0 = empty), shard g's indices offset by v0[g]
+    (int32 device tensor [G] or None).  Returns (idx [R][s], val [R][s])."""
+    G, R, c = idxs.shape
+    _need(vals, "vals", torch.float32, (G, R, c))
+    _need(idxs, "idxs", torch.int32, (G, R, c))
+    return _merge(_ptr(vals), _ptr(idxs), R * c, G, R, c, s, v0, out, idxs.device)
+
+
+def medusa_topk_merge_planes(cand, s: int, v0=None, out=None):
+    """As medusa_topk_merge on one int32 buffer cand [G][2][R][c]: plane 0
+    holds the fp32 values' bits, plane 1 the ids (the layout an all-gather
+    of each shard's [values; ids] buffer produces), read in place."""
+    G, two, R, c = cand.shape
+    _need(cand, "cand", torch.int32, (G, 2, R, c))
+    base = cand.data_ptr()
+    return _merge(base, base + 4 * R * c, 2 * R * c, G, R, c, s, v0, out, cand.device)
+
+
 def medusa_build_tree(tree: Tree, root_tok, topk_idx, prefix_len, out=None):
     B = root_tok.shape[0]
     _need(root_tok, "root_tok", torch.int32, (B,))

@@ -166,6 +166,10 @@ int kv_compact_launch(void* k, void* v, const int32_t* L, const int32_t* alen,
 
 // ---------------------------------------------------------------- TMA descriptors
 // Encodes a bf16 tensor map (dims innermost first) with 128-byte swizzling.
+// merge of per-shard top-s candidate lists (csrc/topk.cu)
+int topk_merge_launch(const float* val, const int32_t* idx, long long gs, const int32_t* v0, int G,
+                      int R, int c, int s, int32_t* out_idx, float* out_val, cudaStream_t st);
+
 // sampled next token (csrc/sample.cu)
 int sample_next_launch(const void* vlog, int dtype, const int32_t* alen, const int32_t* anodes,
                        int B, int N, int V, int K, float temperature, uint64_t seed,

@@ -542,6 +542,18 @@ int medusa_kv_compact(void* k_cache, void* v_cache, const int32_t* prefix_len,
                            Lcap, K, dtype, new_len, (cudaStream_t)stream);
 }
 
+int medusa_topk_merge(const float* val, const int32_t* idx, long long shard_stride,
+                      const int32_t* v0, int G, int R, int c, int s, int32_t* out_idx,
+                      float* out_val, void* stream) {
+  if (G < 1 || R < 0 || c < 1 || s < 1 || s > MEDUSA_MAX_S || (long long)G * c > (1LL << 30))
+    return fail(MEDUSA_ERR_INVALID_ARG, "bad shape");
+  if (shard_stride < (long long)R * c) return fail(MEDUSA_ERR_INVALID_ARG, "shard_stride < R * c");
+  if (R == 0) return MEDUSA_OK;
+  if (!val || !idx || !out_idx) return fail(MEDUSA_ERR_INVALID_ARG, "NULL pointer");
+  return topk_merge_launch(val, idx, shard_stride, v0, G, R, c, s, out_idx, out_val,
+                           (cudaStream_t)stream);
+}
+
 int medusa_sample_next(const void* vlogits, int dtype, const int32_t* accept_len,
                        const int32_t* accept_nodes, int B, int N, int V, int K,
                        float temperature, uint64_t seed, uint64_t offset,

@@ -100,7 +100,45 @@ __global__ void __launch_bounds__(kThreads) topk_keys_kernel(const uint64_t* __r
   block_select(k, s, red, idx + row * s, val ? val + row * s : nullptr);
 }
 
+// Candidate lists of G shards: shard g's list for row r is val / idx
+// [g * gs + r * c .. + c) (index < 0: empty slot).  The row's s best by value
+// descending, ties to the lower index; shard g's indices are offset by v0[g]
+// (device array) when v0 is given.
+__global__ void __launch_bounds__(kThreads)
+    topk_merge_kernel(const float* __restrict__ val, const int32_t* __restrict__ idx,
+                      long long gs, const int32_t* __restrict__ v0, int G, int R, int c, int s,
+                      int32_t* __restrict__ out_idx, float* __restrict__ out_val) {
+  // nothing in this kernel runs ahead of its predecessor
+  griddep_launch_dependents();
+  griddep_wait();
+  __shared__ uint64_t red[kThreads / 32];
+  const int row = blockIdx.x;
+  uint64_t k[kSmax];
+#pragma unroll
+  for (int i = 0; i < kSmax; ++i) k[i] = 0ull;
+  uint64_t kth = 0ull;
+  const int C = G * c;
+  for (int t = threadIdx.x; t < C; t += kThreads) {
+    const int g = t / c, j = t - g * c;
+    const size_t o = (size_t)g * (size_t)gs + (size_t)row * c + j;
+    const int i = idx[o];
+    if (i < 0) continue;
+    const uint64_t key = make_key(val[o], (uint32_t)(i + (v0 ? v0[g] : 0)));
+    if (key > kth) topk_insert<kSmax>(k, s, key, kth);
+  }
+  block_select(k, s, red, out_idx + (size_t)row * s, out_val ? out_val + (size_t)row * s : nullptr);
+}
+
 }  // namespace
+
+int topk_merge_launch(const float* val, const int32_t* idx, long long gs, const int32_t* v0, int G,
+                      int R, int c, int s, int32_t* out_idx, float* out_val, cudaStream_t st) {
+  if (R == 0) return MEDUSA_OK;
+  cudaError_t e = launch_pdl(topk_merge_kernel, dim3(R), dim3(kThreads), 0, st, val, idx, gs, v0, G,
+                             R, c, s, out_idx, out_val);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "topk_merge_kernel launch");
+}
 
 int topk_rows_launch(const void* x, int dtype, int R, int V, int s, int32_t* idx, float* val,
                      cudaStream_t st) {
