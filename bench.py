@@ -33,6 +33,8 @@ METRIC = "verify steps/s"
 EVENT_EVERY = 8  # timed steps per step whose heads / attention calls are bracketed by events
 DECODE_STEPS = 128  # chained steps of the decode-loop measurement
 SAMPLE_REPS = 50    # timed calls of the sampled-next-token measurement
+SHARD_REPS = 50     # timed calls per shard count of the vocabulary-sharded heads
+SHARD_COUNTS = (2, 4, 8)
 E2E_GRAPH_STEPS = 8  # end-to-end steps per captured CUDA graph
 
 
@@ -328,8 +330,8 @@ def run_ours(args, cfg, world, rank, local):
 
     # end to end through the public API with host buffers: every step copies
     # its inputs from pinned host memory (the next step's on a copy stream,
-    # overlapped with this step's kernels; the tree K/V slots on the compute
-    # stream) and reads its results back
+    # overlapped with this step's kernels, its tree K/V slots ahead of the
+    # rest) and reads its results back
     io = PipelinedHostIO(st)
     io.capture(E2E_GRAPH_STEPS)     # E2E_GRAPH_STEPS steps per graph launch
     Ke = E2E_GRAPH_STEPS * max(2, K // (8 * E2E_GRAPH_STEPS))
@@ -362,6 +364,53 @@ def run_ours(args, cfg, world, rank, local):
     s1.record(stream)
     torch.cuda.synchronize(dev)
     sample_ms = s0.elapsed_time(s1) / SAMPLE_REPS
+
+    # Vocabulary-sharded heads, one rank's share of the work for G shards:
+    # the replicated first projection, the second over the first (largest)
+    # W2 shard, and the merge of G candidate lists, CUDA events around
+    # SHARD_REPS calls.  The all-gather between them needs G GPUs and is not
+    # in this figure.
+    from medusa_head_speculative_02_b200.sharded import shard_offsets, shard_w2, vocab_shard
+    sharded = {}
+    R = cfg.B * cfg.K
+    elt = 4 if cfg.dtype == "f32" else 2
+    for G in SHARD_COUNTS:
+        v0, v1 = vocab_shard(cfg.V, G, 0)
+        if v1 - v0 < cfg.s:
+            continue
+        W2g = shard_w2(st.x["W2"], G, 0)
+        cand = torch.zeros(G, 2, R, cfg.s, dtype=torch.int32, device=dev)
+        offs = torch.tensor(shard_offsets(cfg.V, G), dtype=torch.int32, device=dev)
+        ws = torch.empty(max(256, _api.heads_workspace_size(cfg.B, cfg.d, v1 - v0, cfg.K, cfg.s,
+                                                            st.x["h"].dtype)),
+                         dtype=torch.uint8, device=dev)
+        outs = (torch.empty(R, cfg.s, dtype=torch.int32, device=dev),
+                torch.empty(R, cfg.s, dtype=torch.float32, device=dev))
+        pl = (None, cand[0, 1].view(cfg.B, cfg.K, cfg.s),
+              cand[0, 0].view(torch.float32).view(cfg.B, cfg.K, cfg.s))
+
+        def one_rank():
+            _api.medusa_heads_forward(st.x["h"], st.x["W1"], st.x["b1"], W2g, s=cfg.s,
+                                      want_logits=False, out=pl, ws=ws)
+            _api.medusa_topk_merge_planes(cand, cfg.s, offs, out=outs)
+
+        one_rank()
+        cand[1:] = cand[0]          # every shard's list slot holds a real list
+        for _ in range(3):
+            one_rank()
+        torch.cuda.synchronize(dev)
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(SHARD_REPS):
+            one_rank()
+        g1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = g0.elapsed_time(g1) / SHARD_REPS
+        nbytes = st.heads_bytes() - elt * cfg.K * (cfg.V - (v1 - v0)) * cfg.d
+        sharded[str(G)] = {"avg_ms": ms, "algorithmic_bytes": nbytes,
+                           "achieved": nbytes / (ms / 1e3) / 1e9, "vocab_rows": v1 - v0}
+        del W2g, cand, ws
+    torch.cuda.empty_cache()
 
     # Multi-step decode: the next token of each step is the next root and its
     # new lengths the next prefix lengths; one step is captured into a CUDA
@@ -436,7 +485,14 @@ def run_ours(args, cfg, world, rank, local):
                                             "achieved": sample_bytes / (sample_ms / 1e3) / 1e9,
                                             "unit": "GB/s",
                                             "note": "one verify row per sequence; "
-                                                    "latency-bound at small batch"}},
+                                                    "latency-bound at small batch"},
+                            "sharded_heads": {"per_shard_count": sharded, "unit": "GB/s",
+                                              "note": "one rank's heads for G vocabulary "
+                                                      "shards: replicated first projection, "
+                                                      "its W2 rows, merge of G candidate "
+                                                      "lists; the all-gather of G * B * K * s "
+                                                      "* 8 bytes between them is not "
+                                                      "included (needs G GPUs)"}},
                 "decode_loop": ({"steps": DECODE_STEPS, "cuda_graph": True,
                                  "steps_per_s": dec["value"],
                                  "tokens_per_s": dec["value"] * cfg.B * (1.0 + dec_alen),
@@ -448,9 +504,9 @@ def run_ours(args, cfg, world, rank, local):
                         "h2d_bytes_per_step": io.h2d_bytes(),
                         "d2h_bytes_per_step": io.d2h_bytes(), "steps": Ke,
                         "copies": "pinned host -> device every step; the next step's "
-                                  "hidden state, queries, verify logits, roots and lengths "
-                                  "on a copy stream overlapping this step, the tree K/V "
-                                  "slots on the compute stream",
+                                  "tree K/V slots, then its hidden state, queries, verify "
+                                  "logits, roots and lengths, on a copy stream overlapping "
+                                  "this step",
                         "launch": f"API calls and copies of {E2E_GRAPH_STEPS} steps captured "
                                   f"once into a CUDA graph, replayed"},
                 "gpu_launches": st.launches_per_step() * K,
