@@ -440,6 +440,10 @@ def run_ours(args, cfg, world, rank, local):
     del loop
 
     peaks = measured_peaks()
+    attn_chunks = _api.attention_chunks(st.tree, cfg.B, cfg.Hq, cfg.Hkv, cfg.dh, cfg.Lcap,
+                                        cfg.torch_dtype)
+    attn_launches = _api.attention_launches(st.tree, cfg.B, cfg.Hq, cfg.Hkv, cfg.dh, cfg.Lcap,
+                                            cfg.torch_dtype)
     sample_bytes = cfg.B * cfg.V * (4 if cfg.dtype == "f32" else 2)
     hb = st.heads_bytes()
     ab = st.attention_bytes()
@@ -479,7 +483,9 @@ def run_ours(args, cfg, world, rank, local):
                              "algorithmic_bytes": hb, "avg_ms": heads_ms},
                 "kernels": {"tree_attention": {"achieved": attn_gbs, "unit": "GB/s",
                                                "frac": attn_gbs / peaks["hbm_gbs"],
-                                               "algorithmic_bytes": ab, "avg_ms": attn_ms},
+                                               "algorithmic_bytes": ab, "avg_ms": attn_ms,
+                                               "key_chunks": attn_chunks,
+                                               "launches": attn_launches},
                             "sample_next": {"avg_ms": sample_ms, "temperature": 0.7,
                                             "algorithmic_bytes": sample_bytes,
                                             "achieved": sample_bytes / (sample_ms / 1e3) / 1e9,

@@ -198,12 +198,23 @@ size_t medusa_tree_attention_workspace_size(const medusa_tree_t* tree, int B,
 
 /*
  * Number of key chunks medusa_tree_attention splits each (sequence, kv-head)
- * into for these sizes on the current device (>= 1; with more than one, a
- * combine kernel follows the attention kernel).  Negative status on bad
- * arguments.  Introspection only (used to count kernel launches).
+ * into for these sizes on the current device (>= 1).  With more than one,
+ * the chunks' partial results are merged either inside the attention kernel
+ * (bf16, dh = 128, at most 8 chunks, and every thread-block cluster of the
+ * chunks of one query tile resident on the device at once: the chunks merge
+ * through distributed shared memory) or by a combine kernel that follows it.
+ * Negative status on bad arguments.  Introspection only.
  */
 int medusa_tree_attention_chunks(const medusa_tree_t* tree, int B, int Hq,
                                  int Hkv, int dh, int Lcap, int dtype);
+
+/*
+ * Number of kernels one medusa_tree_attention call with these sizes launches
+ * on the current device (0 for B = 0, else 1 or 2).  Negative status on bad
+ * arguments.  Introspection only (used to count kernel launches).
+ */
+int medusa_tree_attention_launches(const medusa_tree_t* tree, int B, int Hq,
+                                   int Hkv, int dh, int Lcap, int dtype);
 
 int medusa_tree_attention(const void* q, const void* k_cache,
                           const void* v_cache, const int32_t* prefix_len,

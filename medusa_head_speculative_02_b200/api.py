@@ -211,6 +211,14 @@ def attention_chunks(tree: Tree, B, Hq, Hkv, dh, Lcap, dtype: torch.dtype) -> in
     return n
 
 
+def attention_launches(tree: Tree, B, Hq, Hkv, dh, Lcap, dtype: torch.dtype) -> int:
+    """Kernels one medusa_tree_attention call launches on the current device."""
+    n = int(L.lib().medusa_tree_attention_launches(tree.handle, B, Hq, Hkv, dh, Lcap, _DT[dtype]))
+    if n < 0:
+        L.check(n, "medusa_tree_attention_launches")
+    return n
+
+
 def medusa_tree_attention(q, k_cache, v_cache, prefix_len, tree: Tree, scale: float, out=None,
                           ws=None):
     B, N, Hq, dh = q.shape

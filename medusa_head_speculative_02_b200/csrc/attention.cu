@@ -258,6 +258,15 @@ int attention_chunks(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int L
   return make_plan(t, B, Hq, Hkv, dh, Lcap).chunks;
 }
 
+int attention_launches(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lcap, int dtype) {
+  if (B == 0) return 0;
+  if (attention_tc_eligible(dtype, dh, Hq, Hkv)) {
+    const int P = make_tc_plan(t, B, Hq, Hkv, dh, Lcap).P;
+    return (P <= 1 || attention_tc_fuse(B, Hq, Hkv, t->N, P)) ? 1 : 2;
+  }
+  return 2;  // SIMT kernel and its combine kernel
+}
+
 size_t attention_workspace(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lcap,
                            int dtype) {
   const size_t simt = make_plan(t, B, Hq, Hkv, dh, Lcap).total;
@@ -277,8 +286,9 @@ int attention_launch(const AttnArgs& a, cudaStream_t st) {
     if (a.B == 0) return MEDUSA_OK;
     float* po = (float*)((uint8_t*)a.ws + P.off_o);
     float2* pml = (float2*)((uint8_t*)a.ws + P.off_ml);
-    int rc = attention_tc_run(a, P.P, po, pml, st);
-    if (rc || P.P == 1) return rc;
+    const bool fuse = attention_tc_fuse(a.B, a.Hq, a.Hkv, t->N, P.P);
+    int rc = attention_tc_run(a, P.P, fuse, po, pml, st);
+    if (rc || P.P == 1 || fuse) return rc;
     const int R = t->N * (a.Hq / a.Hkv);
     const int rows = a.B * t->N * a.Hq;
     cudaError_t e = launch_pdl(tree_attn_combine_kernel<__nv_bfloat16, 128>, dim3((rows + 7) / 8),

@@ -33,12 +33,20 @@
 // warp 1 issues the MMAs, warps 2-5 / 6-9 are the softmax warpgroups of key
 // halves 0 / 1; the two warps that share a TMEM lane quadrant meet at a
 // named barrier once per tile.  With one chunk the CTA writes the
-// normalised output; with more it writes unnormalised partials (O, max,
-// sum) for the combine kernel.
+// normalised output.  With more, the chunks of a query tile either form a
+// thread-block cluster (one CTA per chunk, when every cluster of the launch
+// fits on the GPU at once): each CTA stages its unnormalised O rows and
+// (max, sum) in its own shared memory, the K/V rings being free by then, and
+// rank c merges rows [c R/P, (c+1) R/P) of the tile from all ranks through
+// distributed shared memory; or they write the partials to the workspace for
+// the combine kernel.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace medusa {
+namespace cg = cooperative_groups;
 namespace {
 
 constexpr int kThreads = 352;  // K producer, MMA issuer, 2 x 4 softmax warps, V producer
@@ -53,12 +61,20 @@ constexpr size_t kDataBytes = (1 + 2 * kStages) * (size_t)TILE;  // Q | K ring |
 constexpr size_t kXchBytes = 2 * 2 * BM * sizeof(uint16_t);  // row-max exchange
 constexpr size_t SMEM = 1024 + kDataBytes + 256 + kXchBytes;
 constexpr float kRescale = 8.0f;  // log2 of the growth that forces a rescale
+constexpr int kMaxClusterChunks = 8;  // portable cluster size
+// Staged O rows of the cluster merge: fp32, a row stride of DH + 4 floats, so
+// the float4 stores of 8 consecutive rows fall in distinct banks.
+constexpr int OST = DH + 4;
+constexpr size_t kOStage = (size_t)BM * OST * sizeof(float);
+static_assert(kOStage + BM * sizeof(float2) <= 2 * kStages * (size_t)TILE,
+              "staged O rows and (max, sum) fit in the K/V rings");
 static_assert(MEDUSA_MAX_N == 256, "ancestor words are selected for at most 4 x 64 nodes");
 
 struct TcAttnParams {
   const int32_t* L;
   const uint32_t* anc;
   int B, N, W, Hq, Hkv, G, Lcap, R, P, mtiles;
+  int fuse;      // 1: the P chunks of a query tile are one cluster and merge in the kernel
   float qscale;  // softmax scale * log2(e)
   __nv_bfloat16* out;
   float* po;
@@ -158,6 +174,55 @@ __device__ __forceinline__ float max64(const float (&v)[64]) {
                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
 }
 
+// Merge of the P chunks of query tile qt of (sequence b, kv-head kvh) by the
+// cluster they form (rank = chunk): every rank has staged its unnormalised O
+// rows (so, row stride OST) and their (max, sum) in base 2 (sml; max = -inf:
+// no visible key in that chunk) in its own shared memory.  Rank c takes rows
+// [c per, (c+1) per) of the tile, one warp per row: the row max M over the
+// chunks, weights 2^(m_c - M), and out = sum_c w_c O_c / sum_c w_c l_c as
+// bf16 (0 for a row that sees no key).  Every thread of every rank calls it
+// exactly once.
+__device__ __forceinline__ void cluster_merge(float* so, float2* sml, int qt, int b, int kvh, int P,
+                                              int R, int G, int N, int Hq,
+                                              __nv_bfloat16* __restrict__ out) {
+  cg::cluster_group cl = cg::this_cluster();
+  cl.sync();  // every rank's partial rows are in its shared memory
+  const int rank = (int)cl.block_rank();
+  const int live = min(BM, R - qt * BM);
+  const int per = (live + P - 1) / P;
+  const int r0 = rank * per, r1 = min(live, r0 + per);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int r = r0 + warp; r < r1; r += kThreads / 32) {
+    const float2 ml = lane < P ? cl.map_shared_rank(sml, lane)[r] : make_float2(-INFINITY, 0.f);
+    float M = ml.x;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float w = (lane < P && ml.x != -INFINITY) ? exp2f(ml.x - M) : 0.f;
+    float Ls = w * ml.y;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = 0; c < P; ++c) {
+      const float wc = __shfl_sync(0xffffffffu, w, c);
+      if (wc != 0.f) {
+        const float4 o = reinterpret_cast<const float4*>(cl.map_shared_rank(so, c) + (size_t)r * OST)[lane];
+        acc.x = fmaf(wc, o.x, acc.x);
+        acc.y = fmaf(wc, o.y, acc.y);
+        acc.z = fmaf(wc, o.z, acc.z);
+        acc.w = fmaf(wc, o.w, acc.w);
+      }
+    }
+    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+    const int grow = qt * BM + r;
+    const int node = grow / G, g = grow - node * G;
+    __nv_bfloat16* dst = out + (((size_t)b * N + node) * Hq + (size_t)kvh * G + g) * DH + lane * 4;
+    __align__(8) __nv_bfloat162 h[2] = {__floats2bfloat162_rn(acc.x * inv, acc.y * inv),
+                                        __floats2bfloat162_rn(acc.z * inv, acc.w * inv)};
+    *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(h);
+  }
+  cl.sync();  // every rank stays resident until the others have read its rows
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
@@ -213,6 +278,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int T = rg.n_pre + rg.n_tree;
 
   if (T == 0) {  // nothing to attend to in this chunk
+    if (p.fuse) {
+      float2* sml = (float2*)(sm + TILE + kOStage);
+      if (threadIdx.x < BM) sml[threadIdx.x] = make_float2(-INFINITY, 0.f);
+      griddep_launch_dependents();
+      cluster_merge((float*)(sm + TILE), sml, qt, b, kvh, p.P, p.R, p.G, p.N, p.Hq, p.out);
+      return;
+    }
     if (threadIdx.x < BM) {
       const int grow = qt * BM + threadIdx.x;
       if (grow < p.R) write_row<DH>(p, b, kvh, chunk, grow, 0, -INFINITY, 0.f, nullptr, true);
@@ -473,7 +545,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
     }
     const bool bad = bar_red_or(2, 256, !ok || *abort_flag);
-    if (!bad && warp_live) {
+    if (p.fuse) {
+      // stage this chunk's rows for the cluster merge: every MMA has completed
+      // and every K/V load has landed, so the rings are free
+      float* so = (float*)sK;
+      float2* sml = (float2*)(sK + kOStage);
+      const bool have = !bad && warp_live && row_ok && m_used != -INFINITY;
+      float Ls = 0.f;
+      if (!bad && warp_live) {
+        tc_fence_after();
+        Ls = l + tmem_ld1(tmem + lane_base + (uint32_t)(hf ^ 1));
+#pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 32) {
+          float a[32];
+          tmem_ld32(tO + (uint32_t)c0, a);
+          if (have) {
+            float4* dst = reinterpret_cast<float4*>(so + (size_t)r * OST + hf * 64 + c0);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(a[4 * e], a[4 * e + 1], a[4 * e + 2], a[4 * e + 3]);
+          }
+        }
+      }
+      if (hf == 0) sml[r] = have ? make_float2(m_used, Ls) : make_float2(-INFINITY, 0.f);
+    } else if (!bad && warp_live) {
       tc_fence_after();
       const float Ls = l + tmem_ld1(tmem + lane_base + (uint32_t)(hf ^ 1));
       const int cb = hf * 64;
@@ -498,6 +593,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  if (p.fuse)
+    cluster_merge((float*)sK, (float2*)(sK + kOStage), qt, b, kvh, p.P, p.R, p.G, p.N, p.Hq,
+                  p.out);
+}
+
+std::atomic<bool> g_smem_attr[64];  // per device: the kernel's shared-memory limit raised
+
+// Clusters of P CTAs of this kernel that can be resident at once on the
+// current device (0 when the query fails), cached per device and P.
+int max_active_clusters(int P) {
+  static std::atomic<int> cache[64][kMaxClusterChunks + 1];
+  int dev = 0;
+  if (P < 1 || P > kMaxClusterChunks || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return 0;
+  }
+  const int v = cache[dev][P].load(std::memory_order_relaxed);
+  if (v) return v - 1;
+  if (ensure_max_smem(tree_attn_tc_kernel, (int)SMEM, g_smem_attr,
+                      "cudaFuncSetAttribute(tree_attn_tc_kernel)"))
+    return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, P, 1);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = SMEM;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = P;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, (void*)tree_attn_tc_kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();  // not an error of the caller's stream: merge with the combine kernel
+    return 0;
+  }
+  cache[dev][P].store(n + 1, std::memory_order_relaxed);
+  return n;
 }
 
 }  // namespace
@@ -520,7 +654,16 @@ int attention_tc_chunks(int B, int Hq, int Hkv, int N, int Lcap) {
   return (int)P;
 }
 
-int attention_tc_run(const AttnArgs& a, int P, float* po, float2* pml, cudaStream_t st) {
+bool attention_tc_fuse(int B, int Hq, int Hkv, int N, int P) {
+  if (P < 2 || P > kMaxClusterChunks || B <= 0) return false;
+  const long long R = (long long)N * (Hq / Hkv);
+  const long long units = (long long)B * Hkv * ((R + BM - 1) / BM);
+  const int n = max_active_clusters(P);
+  return n > 0 && units <= n;
+}
+
+int attention_tc_run(const AttnArgs& a, int P, bool fuse, float* po, float2* pml,
+                     cudaStream_t st) {
   const medusa_tree* t = a.tree;
   const int G = a.Hq / a.Hkv;
   const int R = t->N * G;
@@ -542,8 +685,7 @@ int attention_tc_run(const AttnArgs& a, int P, float* po, float2* pml, cudaStrea
     rc = make_tmap_bf16(&mV, a.v, 3, dims, strides, box);
     if (rc) return rc;
   }
-  static std::atomic<bool> attr_done[64];
-  int rc = ensure_max_smem(tree_attn_tc_kernel, (int)SMEM, attr_done,
+  int rc = ensure_max_smem(tree_attn_tc_kernel, (int)SMEM, g_smem_attr,
                            "cudaFuncSetAttribute(tree_attn_tc_kernel)");
   if (rc) return rc;
   TcAttnParams p;
@@ -559,12 +701,33 @@ int attention_tc_run(const AttnArgs& a, int P, float* po, float2* pml, cudaStrea
   p.R = R;
   p.P = P;
   p.mtiles = mtiles;
+  p.fuse = (fuse && P >= 2 && P <= kMaxClusterChunks) ? 1 : 0;
   p.qscale = a.scale * 1.4426950408889634f;
   p.out = (__nv_bfloat16*)a.out;
   p.po = po;
   p.pml = pml;
   dim3 grid(mtiles, P, a.B * a.Hkv);
-  cudaError_t e = launch_pdl(tree_attn_tc_kernel, grid, dim3(kThreads), SMEM, st, mQ, mK, mV, p);
+  cudaError_t e;
+  if (p.fuse) {
+    // the P chunks of a query tile (grid y) are one cluster
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = P;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    e = cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel, mQ, mK, mV, p);
+  } else {
+    e = launch_pdl(tree_attn_tc_kernel, grid, dim3(kThreads), SMEM, st, mQ, mK, mV, p);
+  }
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "tree_attn_tc_kernel launch");
 }

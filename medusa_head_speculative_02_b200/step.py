@@ -17,9 +17,8 @@ from .synthetic import MedusaConfig, gen_inputs, plant_verify_logits
 
 # kernels this library launches per call
 # (heads: stage-1 GEMM, SiLU epilogue, stage-2 GEMM, top-s merge; attention:
-# the attention kernel, plus a combine kernel when it splits the keys into
-# chunks)
-LAUNCHES = {"heads": 4, "build_tree": 1, "tree_attention": 1, "accept": 2, "kv_compact": 1}
+# one or two, asked of the library, see launches_per_step)
+LAUNCHES = {"heads": 4, "build_tree": 1, "accept": 2, "kv_compact": 1}
 
 
 class VerifyStep:
@@ -100,9 +99,9 @@ class VerifyStep:
     def launches_per_step(self) -> int:
         c = self.cfg
         n_acc = 2 if c.accept == "both" else 1
-        chunks = api.attention_chunks(self.tree, c.B, c.Hq, c.Hkv, c.dh, c.Lcap, c.torch_dtype)
-        return (LAUNCHES["heads"] + LAUNCHES["build_tree"] + LAUNCHES["tree_attention"] +
-                (1 if chunks > 1 else 0) + n_acc * LAUNCHES["accept"] + LAUNCHES["kv_compact"])
+        attn = api.attention_launches(self.tree, c.B, c.Hq, c.Hkv, c.dh, c.Lcap, c.torch_dtype)
+        return (LAUNCHES["heads"] + LAUNCHES["build_tree"] + attn + n_acc * LAUNCHES["accept"] +
+                LAUNCHES["kv_compact"])
 
     # algorithmic bytes --------------------------------------------------------
     def heads_bytes(self) -> int:

@@ -1,0 +1,66 @@
+"""GPU: tree attention whose keys are split into 2 to 8 chunks merged inside
+the kernel (the chunks of a query tile run as one thread-block cluster and
+merge through distributed shared memory), against the fp64 oracle on every
+output row (max-abs 2e-2): MHA and GQA, one and several query tiles, ragged
+prefixes, chunks that see no key (a short or empty prefix next to a long
+cache), and the launch count the library reports."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import medusa_oracle as O
+from medusa_head_speculative_02_b200 import api
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+ATOL = 2e-2
+
+
+@pytest.mark.parametrize("B,tree,Hq,Hkv,Ls", [
+    (1, (5, 10, 64), 2, 2, [700]),             # 2 chunks
+    (3, (3, 2, 7), 4, 1, [600, 0, 1200]),      # GQA, an empty prefix
+    (1, (5, 10, 64), 4, 4, [2048]),            # 7B-like rows, 5 chunks
+    (2, (5, 10, 64), 8, 2, [50, 3000]),        # 2 query tiles, keyless chunks
+    (1, (4, 4, 32), 2, 2, [4000]),             # 8 chunks
+    (2, (5, 8, 128), 8, 2, [1000, 777]),       # 4 query tiles
+])
+def test_fused_chunk_merge_matches_oracle(B, tree, Hq, Hkv, Ls):
+    K, s, N = tree
+    dh = 128
+    Lcap = max(Ls) + N + 3
+    g = torch.Generator(device=DEV).manual_seed(B * 1000 + Lcap)
+    q = torch.randn(B, N, Hq, dh, generator=g, device=DEV).bfloat16()
+    kc = torch.randn(B, Lcap, Hkv, dh, generator=g, device=DEV).bfloat16()
+    vc = torch.randn(B, Lcap, Hkv, dh, generator=g, device=DEV).bfloat16()
+    L = torch.tensor(Ls, dtype=torch.int32, device=DEV)
+    t = api.Tree(K, s, N)
+    P = api.attention_chunks(t, B, Hq, Hkv, dh, Lcap, torch.bfloat16)
+    assert 2 <= P <= 8
+    assert api.attention_launches(t, B, Hq, Hkv, dh, Lcap, torch.bfloat16) == 1
+    scale = 1.0 / math.sqrt(dh)
+    out = api.medusa_tree_attention(q, kc, vc, L, t, scale)
+    torch.cuda.synchronize()
+    ref = O.tree_attention(q, kc, vc, L, O.tree_plan(K, s, N), scale)
+    err = np.abs(out.double().cpu().numpy() - ref).max()
+    assert err <= ATOL, err
+    assert api.device_status() == 0
+
+
+def test_fused_merge_is_repeatable_and_leaves_no_state():
+    """Two calls on the same inputs give the same bits (nothing carried over
+    between calls), and a call on other inputs in between changes nothing."""
+    B, (K, s, N), Hq, Hkv, dh = 2, (5, 10, 64), 8, 2, 128
+    Lcap = 3000 + N
+    g = torch.Generator(device=DEV).manual_seed(9)
+    mk = lambda *shape: torch.randn(*shape, generator=g, device=DEV).bfloat16()
+    q, kc, vc = mk(B, N, Hq, dh), mk(B, Lcap, Hkv, dh), mk(B, Lcap, Hkv, dh)
+    q2, kc2, vc2 = mk(B, N, Hq, dh), mk(B, Lcap, Hkv, dh), mk(B, Lcap, Hkv, dh)
+    L = torch.tensor([2900, 123], dtype=torch.int32, device=DEV)
+    t = api.Tree(K, s, N)
+    a = api.medusa_tree_attention(q, kc, vc, L, t, 0.1).clone()
+    api.medusa_tree_attention(q2, kc2, vc2, L, t, 0.1)
+    b = api.medusa_tree_attention(q, kc, vc, L, t, 0.1)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
