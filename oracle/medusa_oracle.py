@@ -36,7 +36,10 @@ the last accepted node's row; tree positions are prefix_len + depth; with
 one temperature per head, the candidates of depth D are verified at the
 temperature of head D; the
 sampled next token is drawn from the last accepted node's row by Gumbel-max
-with SplitMix64 noise keyed by (seed, call offset, sequence, vocab index).
+with SplitMix64 noise keyed by (seed, call offset, sequence, vocab index);
+candidate lists of vocabulary shards merge in the top-s order of the whole
+row (value desc, global id asc), so a merge of per-shard top-s lists equals
+the top-s of the unsplit row.
 
 Parity: every function here is pinned by tests/test_oracle_pins.py against
 closed forms, library routines or brute force (see each docstring).
