@@ -444,6 +444,8 @@ def run_ours(args, cfg, world, rank, local):
                                         cfg.torch_dtype)
     attn_launches = _api.attention_launches(st.tree, cfg.B, cfg.Hq, cfg.Hkv, cfg.dh, cfg.Lcap,
                                             cfg.torch_dtype)
+    attn_tiles = _api.attention_tiles_per_cta(st.tree, cfg.B, cfg.Hq, cfg.Hkv, cfg.dh, cfg.Lcap,
+                                              cfg.torch_dtype)
     sample_bytes = cfg.B * cfg.V * (4 if cfg.dtype == "f32" else 2)
     hb = st.heads_bytes()
     ab = st.attention_bytes()
@@ -485,6 +487,7 @@ def run_ours(args, cfg, world, rank, local):
                                                "frac": attn_gbs / peaks["hbm_gbs"],
                                                "algorithmic_bytes": ab, "avg_ms": attn_ms,
                                                "key_chunks": attn_chunks,
+                                               "query_tiles_per_cta": attn_tiles,
                                                "launches": attn_launches},
                             "sample_next": {"avg_ms": sample_ms, "temperature": 0.7,
                                             "algorithmic_bytes": sample_bytes,

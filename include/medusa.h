@@ -216,6 +216,18 @@ int medusa_tree_attention_chunks(const medusa_tree_t* tree, int B, int Hq,
 int medusa_tree_attention_launches(const medusa_tree_t* tree, int B, int Hq,
                                    int Hkv, int dh, int Lcap, int dtype);
 
+/*
+ * 128-row query tiles one CTA of medusa_tree_attention takes for these sizes
+ * on the current device: 2 when the keys are not split, a (sequence,
+ * kv-head) has at least two query tiles and pairing them saves enough waves
+ * of CTAs on the device (both tiles then share every K/V tile the CTA
+ * stages), else 1.
+ * Negative status on bad arguments.  Introspection only.
+ */
+int medusa_tree_attention_tiles_per_cta(const medusa_tree_t* tree, int B,
+                                        int Hq, int Hkv, int dh, int Lcap,
+                                        int dtype);
+
 int medusa_tree_attention(const void* q, const void* k_cache,
                           const void* v_cache, const int32_t* prefix_len,
                           const medusa_tree_t* tree, int B, int Hq, int Hkv,

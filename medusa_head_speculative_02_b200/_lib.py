@@ -38,6 +38,7 @@ SIGNATURES = {
     "medusa_tree_attention_workspace_size": (csz, [vp, ci, ci, ci, ci, ci]),
     "medusa_tree_attention_chunks": (ci, [vp, ci, ci, ci, ci, ci, ci]),
     "medusa_tree_attention_launches": (ci, [vp, ci, ci, ci, ci, ci, ci]),
+    "medusa_tree_attention_tiles_per_cta": (ci, [vp, ci, ci, ci, ci, ci, ci]),
     "medusa_tree_attention": (ci, [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp, vp, csz,
                                    vp]),
     "medusa_accept_workspace_size": (csz, [vp, ci, ci]),

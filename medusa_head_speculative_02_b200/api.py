@@ -211,6 +211,15 @@ def attention_chunks(tree: Tree, B, Hq, Hkv, dh, Lcap, dtype: torch.dtype) -> in
     return n
 
 
+def attention_tiles_per_cta(tree: Tree, B, Hq, Hkv, dh, Lcap, dtype: torch.dtype) -> int:
+    """128-row query tiles one attention CTA takes (1 or 2)."""
+    n = int(L.lib().medusa_tree_attention_tiles_per_cta(tree.handle, B, Hq, Hkv, dh, Lcap,
+                                                         _DT[dtype]))
+    if n < 1:
+        L.check(n, "medusa_tree_attention_tiles_per_cta")
+    return n
+
+
 def attention_launches(tree: Tree, B, Hq, Hkv, dh, Lcap, dtype: torch.dtype) -> int:
     """Kernels one medusa_tree_attention call launches on the current device."""
     n = int(L.lib().medusa_tree_attention_launches(tree.handle, B, Hq, Hkv, dh, Lcap, _DT[dtype]))

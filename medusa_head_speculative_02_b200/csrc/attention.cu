@@ -258,6 +258,13 @@ int attention_chunks(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int L
   return make_plan(t, B, Hq, Hkv, dh, Lcap).chunks;
 }
 
+int attention_tiles_per_cta(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lcap,
+                            int dtype) {
+  if (!attention_tc_eligible(dtype, dh, Hq, Hkv)) return 1;
+  const int P = make_tc_plan(t, B, Hq, Hkv, dh, Lcap).P;
+  return attention_tc_pair(B, Hq, Hkv, t->N, P) ? 2 : 1;
+}
+
 int attention_launches(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lcap, int dtype) {
   if (B == 0) return 0;
   if (attention_tc_eligible(dtype, dh, Hq, Hkv)) {

@@ -598,7 +598,378 @@ __global__ void __launch_bounds__(kThreads, 1)
                   p.out);
 }
 
+// ---------------------------------------------------------------------------
+// Two query tiles per CTA.  With one key chunk and at least two 128-row query
+// tiles per (sequence, kv-head), a CTA takes tiles 2x and 2x+1 (the second
+// may lie past the last row: computed, never written) and both read every
+// K/V tile it stages.  TMEM: S/P of tile a | S/P of tile b | O of a | O of b.
+// One softmax warpgroup per tile, so each works on its tile while the
+// tensor pipe runs the other tile's MMAs.  S_q(t) reuses the S/P columns of
+// tile q, so it waits for P.V_q(t-1).
+constexpr int kPairKStages = 3, kPairVStages = 2;
+constexpr size_t kPairData = (2 + kPairKStages + kPairVStages) * (size_t)TILE;
+constexpr size_t SMEM_PAIR = 1024 + kPairData + 256;
+static_assert(SMEM_PAIR <= 227 * 1024, "shared memory of the two-tile kernel");
+
+// mask_half with the ancestor words of the row's node read from memory (two
+// words, only for the tree tiles), so the kernel keeps no per-tile word sets
+// in registers.
+__device__ __forceinline__ void mask_half_mem(float (&v)[64], int j, int hf, const Range& rg,
+                                              int N, int W, const uint32_t* __restrict__ anc_row) {
+  if (j < rg.n_pre) {
+    const int lim = rg.k_hi - (rg.k_lo + j * BN + hf * 64);
+    if (lim < 64) {
+#pragma unroll
+      for (int c = 0; c < 64; ++c) v[c] = (c < lim) ? v[c] : -INFINITY;
+    }
+  } else {
+    const int q = 2 * (j - rg.n_pre) + hf;  // nodes 64q .. 64q+63
+    const uint32_t w0 = (2 * q < W) ? __ldg(anc_row + 2 * q) : 0u;
+    const uint32_t w1 = (2 * q + 1 < W) ? __ldg(anc_row + 2 * q + 1) : 0u;
+    const int nvalid = N - q * 64;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) {
+      const uint32_t word = c < 32 ? w0 : w1;
+      const bool vis = c < nvalid && ((word >> (c & 31)) & 1u);
+      v[c] = vis ? v[c] : -INFINITY;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    tree_attn_tc_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
+                             const __grid_constant__ CUtensorMap tmK,
+                             const __grid_constant__ CUtensorMap tmV, const TcAttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+
+  griddep_wait();  // prefix lengths and the K/V cache may come from the kernel ahead
+  const int qpair = blockIdx.x, bk = blockIdx.z;
+  const int rank = bk / p.Hkv, kvh = bk - rank * p.Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* sQ = sm;  // tile a | tile b
+  uint8_t* sK = sm + 2 * TILE;
+  uint8_t* sV = sK + kPairKStages * TILE;
+  uint64_t* bars = (uint64_t*)(sm + kPairData);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;                  // [kPairKStages]
+  uint64_t* k_empty = k_full + kPairKStages;    // [kPairKStages]
+  uint64_t* v_full = k_empty + kPairKStages;    // [kPairVStages]
+  uint64_t* v_empty = v_full + kPairVStages;    // [kPairVStages]
+  uint64_t* s_full = v_empty + kPairVStages;    // [tile]
+  uint64_t* p_full = s_full + 2;                // [tile]
+  uint64_t* pv_done = p_full + 2;               // [tile]
+  uint64_t* mma_done = pv_done + 2;
+  uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  int* seq_slot = (int*)(tmem_slot + 2);
+
+  int b = rank;  // longest prefix first, as in tree_attn_tc_kernel
+  if (p.B > 1 && p.B <= kThreads) {
+    if ((int)threadIdx.x < p.B) {
+      const int i = threadIdx.x;
+      const int li = p.L[i];
+      int r = 0;
+      for (int j = 0; j < p.B; ++j) {
+        const int lj = p.L[j];
+        r += (lj > li || (lj == li && j < i)) ? 1 : 0;
+      }
+      if (r == rank) *seq_slot = i;
+    }
+    __syncthreads();
+    b = *seq_slot;
+  }
+
+  const int Lb = p.L[b];
+  const bool seq_ok = Lb >= 0 && (long long)Lb + p.N <= p.Lcap;
+  const Range rg = chunk_range(p, Lb, 0, seq_ok);
+  const int T = rg.n_pre + rg.n_tree;
+  const int qt0 = 2 * qpair;  // tile a; tile b = qt0 + 1
+
+  if (T == 0) {
+    for (int q = 0; q < 2; ++q) {
+      const int grow = (qt0 + q) * BM + (int)threadIdx.x;
+      if ((int)threadIdx.x < BM && grow < p.R)
+        write_row<DH>(p, b, kvh, 0, grow, 0, -INFINITY, 0.f, nullptr, true);
+    }
+    return;
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < kPairKStages; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < kPairVStages; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);  // the tile's softmax warps
+      mbar_init(&pv_done[i], 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    __syncwarp();
+    tmem_alloc(tmem_slot, 512);  // S/P a | S/P b | O a | O b
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  griddep_launch_dependents();  // TMEM taken: the next kernel may be scheduled
+
+  if (warp == 0 || warp == kVWarp) {
+    // ---------------------------------------------------------------- TMA producers
+    if (lane == 0) {
+      const bool isK = warp == 0;
+      const uint64_t pol = policy_evict_normal();
+      if (isK) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        mbar_arrive_expect_tx(q_full, 2 * TILE);
+        for (int q = 0; q < 2; ++q) {
+          // rows past the tensor's end read as zero; rows of the next
+          // sequence in tile b of the last pair are computed, never written
+          const int zq = b * p.N + (qt0 + q) * (BM / p.G);
+          tma_load_3d(sQ + q * TILE, &tmQ, q_full, 0, kvh * p.G, zq, pol);
+          tma_load_3d(sQ + q * TILE + HALF, &tmQ, q_full, 64, kvh * p.G, zq, pol);
+        }
+      } else {
+        prefetch_tmap(&tmV);
+      }
+      const int stages = isK ? kPairKStages : kPairVStages;
+      const CUtensorMap* map = isK ? &tmK : &tmV;
+      uint64_t* emp = isK ? k_empty : v_empty;
+      uint64_t* ful = isK ? k_full : v_full;
+      uint8_t* buf = isK ? sK : sV;
+      int issued = 0;
+      for (int j = 0; j < T; ++j) {
+        const int st = j % stages;
+        const int key0 = j < rg.n_pre ? rg.k_lo + j * BN : Lb + (j - rg.n_pre) * BN;
+        const int z = b * p.Lcap + key0;
+        if (!mbar_wait(&emp[st], ((uint32_t)(j / stages) & 1u) ^ 1u, abort_flag)) break;
+        mbar_arrive_expect_tx(&ful[st], TILE);
+        tma_load_3d(buf + st * TILE, map, &ful[st], 0, kvh, z, pol);
+        tma_load_3d(buf + st * TILE + HALF, map, &ful[st], 64, kvh, z, pol);
+        issued = j + 1;
+      }
+      if (issued < T) {
+        // aborted: let the loads already issued land before the CTA exits
+        if (isK) mbar_wait(q_full, 0u, nullptr);
+        for (int j = (issued > stages ? issued - stages : 0); j < issued; ++j)
+          mbar_wait(&ful[j % stages], (uint32_t)(j / stages) & 1u, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = umma_idesc_bf16_f32(BM, BN);
+      const uint32_t idesc_o = umma_idesc_bf16_f32_bmn(BM, DH);
+      auto issue_s = [&](int t, int q) -> bool {
+        const int ks = t % kPairKStages;
+        if (q == 0 && !mbar_wait(&k_full[ks], (uint32_t)(t / kPairKStages) & 1u, abort_flag))
+          return false;
+        // the S/P columns of tile q hold P_q(t-1) until its P.V has run
+        if (t > 0 && !mbar_wait(&pv_done[q], (uint32_t)(t - 1) & 1u, abort_flag)) return false;
+        tc_fence_after();
+        const uint64_t dq = umma_desc_sw128_kmajor(smem_u32(sQ + q * TILE));
+        const uint64_t dk = umma_desc_sw128_kmajor(smem_u32(sK + ks * TILE));
+        const uint32_t dS = tmem + (uint32_t)q * 128u;
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint64_t off = (uint64_t)(((kk >> 2) * HALF + (kk & 3) * 32) >> 4);
+          umma_bf16(dS, dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        if (q == 1) umma_commit(&k_empty[ks]);  // both tiles have read K(t)
+        umma_commit(&s_full[q]);
+        return true;
+      };
+      auto issue_pv = [&](int u, int q) -> bool {
+        const int vs = u % kPairVStages;
+        if (!mbar_wait(&p_full[q], (uint32_t)u & 1u, abort_flag)) return false;
+        if (q == 0 && !mbar_wait(&v_full[vs], (uint32_t)(u / kPairVStages) & 1u, abort_flag))
+          return false;
+        tc_fence_after();
+        const uint64_t dv = umma_desc_sw128(smem_u32(sV + vs * TILE), HALF, 1024u);
+        const uint32_t aP = tmem + (uint32_t)q * 128u;
+        const uint32_t tOq = tmem + 256u + (uint32_t)q * 128u;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16_ts(tOq, aP + (uint32_t)(hf * 64 + kk * 8),
+                         dv + (uint64_t)((hf * 64 * 128 + kk * 16 * 128) >> 4), idesc_o,
+                         (u > 0 || hf > 0 || kk > 0) ? 1u : 0u);
+        if (q == 1) umma_commit(&v_empty[vs]);  // both tiles have read V(u)
+        umma_commit(&pv_done[q]);
+        return true;
+      };
+      // S_a(0), S_b(0), then per key tile t: P.V_a(t), S_a(t+1), P.V_b(t),
+      // S_b(t+1): each tile's next S follows its own P.V, so one tile's
+      // chain (S, softmax, P.V) never waits for the other tile's softmax
+      bool ok = mbar_wait(q_full, 0u, abort_flag) && issue_s(0, 0) && issue_s(0, 1);
+      for (int t = 0; t < T && ok; ++t) {
+        ok = issue_pv(t, 0);
+        if (ok && t + 1 < T) ok = issue_s(t + 1, 0);
+        if (ok) ok = issue_pv(t, 1);
+        if (ok && t + 1 < T) ok = issue_s(t + 1, 1);
+      }
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0u, nullptr);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax warpgroups
+    // warps 2-5: tile a, warps 6-9: tile b; a thread owns one query row and
+    // all 128 keys of every key tile, taken as two 64-key halves under one
+    // running max (lazy rescaling as in tree_attn_tc_kernel).  When the
+    // second half raises the max, the first half's P (already in TMEM) is
+    // rescaled with O.
+    const int q = (warp - 2) >> 2;  // query tile of this warpgroup
+    const int q4 = warp & 3;        // TMEM lane quadrant
+    const int r = q4 * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    const uint32_t tS = tmem + lane_base + (uint32_t)q * 128u;
+    const uint32_t tO = tmem + lane_base + 256u + (uint32_t)q * 128u;
+    const unsigned long long q2 = f2_pack(p.qscale, p.qscale);
+    const int grow = (qt0 + q) * BM + r;
+    const bool row_ok = grow < p.R;
+    const bool live = ((qt0 + q) * BM + q4 * 32) < p.R;  // warp-uniform
+    const uint32_t* anc_row = p.anc + (size_t)min(grow / p.G, p.N - 1) * p.W;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    // Raises the running max to tmax when it grew by more than 2^kRescale:
+    // rescales l, the O row (after P.V(t-1)) and, for the second half, the
+    // first half's P.  Warp-collective (TMEM accesses): every lane calls it.
+    auto maybe_rescale = [&](float tmax, int t, bool p_half0) -> bool {
+      const bool grow_m = tmax > m_used + kRescale;
+      if (!__any_sync(0xffffffffu, grow_m)) return true;
+      float corr = 1.f;
+      if (grow_m) {
+        corr = ex2_approx(m_used - tmax);  // 0 when m_used is -inf
+        m_used = tmax;
+        l *= corr;
+      }
+      if (t > 0) {
+        const bool w_ok = mbar_wait(&pv_done[q], (uint32_t)(t - 1) & 1u, abort_flag);
+        if (!__all_sync(0xffffffffu, w_ok)) return false;
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < DH; c0 += 16) {
+          float o16[16];
+          tmem_ld16(tO + (uint32_t)c0, o16);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o16[e] *= corr;
+          tmem_st16(tO + (uint32_t)c0, o16);
+        }
+      }
+      if (p_half0) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < 32; c0 += 16) {
+          float w16[16];
+          tmem_ld16(tS + (uint32_t)c0, w16);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162*>(&w16[e]);
+            const float2 f = __bfloat1622float2(h2);
+            h2 = __floats2bfloat162_rn(f.x * corr, f.y * corr);
+            w16[e] = *reinterpret_cast<const float*>(&h2);
+          }
+          tmem_st16(tS + (uint32_t)c0, w16);
+        }
+      }
+      return true;
+    };
+    for (int t = 0; t < T && ok; ++t) {
+      const bool good = mbar_wait(&s_full[q], (uint32_t)t & 1u, abort_flag);
+      if (!__all_sync(0xffffffffu, good)) {
+        ok = false;
+        break;
+      }
+      if (live) {
+#pragma unroll 1
+        for (int hf = 0; hf < 2 && ok; ++hf) {
+          float v[64];
+          tc_fence_after();
+          tmem_ld64(tS + (uint32_t)(hf * 64), v);
+          mask_half_mem(v, t, hf, rg, p.N, p.W, anc_row);
+          if (!maybe_rescale(max64(v) * p.qscale, t, hf == 1)) {
+            ok = false;
+            break;
+          }
+          // P = 2^(scale*s - m) in packed pairs (a row with no visible key
+          // yet has m = -inf and only -inf scores, whose exponentials are zeroed)
+          const float moff = (m_used == -INFINITY) ? 0.f : m_used;
+          const unsigned long long m2 = f2_pack(-moff, -moff);
+          unsigned long long sum2[4] = {0ull, 0ull, 0ull, 0ull};
+          uint32_t pk[32];
+#pragma unroll
+          for (int c2 = 0; c2 < 32; ++c2) {
+            float x0, x1, e0, e1;
+            f2_unpack(f2_fma(f2_pack(v[2 * c2], v[2 * c2 + 1]), q2, m2), x0, x1);
+            if ((c2 & 3) == 3) {
+              exp2_fma2(x0, x1, e0, e1);
+            } else {
+              e0 = ex2_approx(x0);
+              e1 = ex2_approx(x1);
+            }
+            sum2[c2 & 3] = f2_add(sum2[c2 & 3], f2_pack(e0, e1));
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
+            pk[c2] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+          tmem_st32(tS + (uint32_t)(hf * 64), pk);  // P over the S columns just read
+          float a0, a1, b0, b1, c0f, c1f, d0, d1;
+          f2_unpack(sum2[0], a0, a1);
+          f2_unpack(sum2[1], b0, b1);
+          f2_unpack(sum2[2], c0f, c1f);
+          f2_unpack(sum2[3], d0, d1);
+          l += ((a0 + a1) + (b0 + b1)) + ((c0f + c1f) + (d0 + d1));
+        }
+        if (!ok) break;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[q]);
+    }
+    // this tile's last P.V complete
+    if (ok && live) {
+      const bool good = mbar_wait(&pv_done[q], (uint32_t)(T - 1) & 1u, abort_flag);
+      ok = __all_sync(0xffffffffu, good);
+    }
+    const bool bad = bar_red_or(2, 256, !ok || *abort_flag);
+    if (!bad && live) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int c0 = 0; c0 < DH; c0 += 32) {
+        float a[32];
+        tmem_ld32(tO + (uint32_t)c0, a);
+        if (row_ok) {
+          if (m_used == -INFINITY)
+            write_row<32>(p, b, kvh, 0, grow, c0, m_used, l, nullptr, c0 == 0);
+          else
+            write_row<32>(p, b, kvh, 0, grow, c0, m_used, l, a, c0 == 0);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 std::atomic<bool> g_smem_attr[64];  // per device: the kernel's shared-memory limit raised
+std::atomic<bool> g_smem_attr_pair[64];
 
 // Clusters of P CTAs of this kernel that can be resident at once on the
 // current device (0 when the query fails), cached per device and P.
@@ -654,6 +1025,20 @@ int attention_tc_chunks(int B, int Hq, int Hkv, int N, int Lcap) {
   return (int)P;
 }
 
+bool attention_tc_pair(int B, int Hq, int Hkv, int N, int P) {
+  if (P != 1 || B <= 0) return false;
+  const long long R = (long long)N * (Hq / Hkv);
+  const long long mtiles = (R + BM - 1) / BM;
+  if (mtiles < 2) return false;
+  // A CTA with two tiles takes about 1.8 times as long per key tile as a CTA
+  // with one (measured on the 8B-GQA and long-context shapes: 2.32-2.35 us
+  // against 1.29-1.34 us), so it pays where it saves enough waves of CTAs.
+  const long long sms = num_sms();
+  const long long w1 = ((long long)B * Hkv * mtiles + sms - 1) / sms;
+  const long long w2 = ((long long)B * Hkv * ((mtiles + 1) / 2) + sms - 1) / sms;
+  return 9 * w2 < 5 * w1;
+}
+
 bool attention_tc_fuse(int B, int Hq, int Hkv, int N, int P) {
   if (P < 2 || P > kMaxClusterChunks || B <= 0) return false;
   const long long R = (long long)N * (Hq / Hkv);
@@ -706,8 +1091,19 @@ int attention_tc_run(const AttnArgs& a, int P, bool fuse, float* po, float2* pml
   p.out = (__nv_bfloat16*)a.out;
   p.po = po;
   p.pml = pml;
-  dim3 grid(mtiles, P, a.B * a.Hkv);
   cudaError_t e;
+  if (attention_tc_pair(a.B, a.Hq, a.Hkv, t->N, P)) {
+    // two query tiles per CTA (one key chunk)
+    rc = ensure_max_smem(tree_attn_tc_pair_kernel, (int)SMEM_PAIR, g_smem_attr_pair,
+                         "cudaFuncSetAttribute(tree_attn_tc_pair_kernel)");
+    if (rc) return rc;
+    p.fuse = 0;
+    e = launch_pdl(tree_attn_tc_pair_kernel, dim3((mtiles + 1) / 2, 1, a.B * a.Hkv),
+                   dim3(kThreads), SMEM_PAIR, st, mQ, mK, mV, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "tree_attn_tc_pair_kernel launch");
+  }
+  dim3 grid(mtiles, P, a.B * a.Hkv);
   if (p.fuse) {
     // the P chunks of a query tile (grid y) are one cluster
     cudaLaunchConfig_t cfg = {};

@@ -133,12 +133,16 @@ size_t attention_workspace(const medusa_tree* t, int B, int Hq, int Hkv, int dh,
 int attention_launch(const AttnArgs& a, cudaStream_t st);
 int attention_chunks(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lcap, int dtype);
 int attention_launches(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lcap, int dtype);
+int attention_tiles_per_cta(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lcap,
+                            int dtype);
 // tcgen05 path (bf16, dh = 128, GQA group dividing 128)
 bool attention_tc_eligible(int dtype, int dh, int Hq, int Hkv);
 int attention_tc_chunks(int B, int Hq, int Hkv, int N, int Lcap);
 // true when the P key chunks of every query tile run as one thread-block
 // cluster, all clusters resident at once, and merge inside the kernel
 bool attention_tc_fuse(int B, int Hq, int Hkv, int N, int P);
+// true when each CTA takes two query tiles of a (sequence, kv-head) (one key chunk)
+bool attention_tc_pair(int B, int Hq, int Hkv, int N, int P);
 int attention_tc_run(const AttnArgs& a, int P, bool fuse, float* po, float2* pml,
                      cudaStream_t st);
 

@@ -415,6 +415,13 @@ int medusa_tree_attention_chunks(const medusa_tree_t* tree, int B, int Hq, int H
   return attention_chunks(tree, B, Hq, Hkv, dh, Lcap, dtype);
 }
 
+int medusa_tree_attention_tiles_per_cta(const medusa_tree_t* tree, int B, int Hq, int Hkv,
+                                        int dh, int Lcap, int dtype) {
+  if (!tree || B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || Lcap < tree->N || !dtype_ok(dtype))
+    return fail(MEDUSA_ERR_INVALID_ARG, "bad attention shape");
+  return attention_tiles_per_cta(tree, B, Hq, Hkv, dh, Lcap, dtype);
+}
+
 int medusa_tree_attention_launches(const medusa_tree_t* tree, int B, int Hq, int Hkv, int dh,
                                    int Lcap, int dtype) {
   if (!tree || B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || Lcap < tree->N || !dtype_ok(dtype))

@@ -64,3 +64,39 @@ def test_fused_merge_is_repeatable_and_leaves_no_state():
     b = api.medusa_tree_attention(q, kc, vc, L, t, 0.1)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------- two query tiles per CTA
+@pytest.mark.parametrize("B,tree,Hq,Hkv,Ls", [
+    # GQA 4: 4 query tiles per (sequence, kv-head), 512 single-tile CTAs
+    (16, (5, 8, 128), 32, 8, [50, 400, 120, 333, 7, 260, 199, 380, 0, 64, 128, 129, 255, 256,
+                              300, 1]),
+    # GQA 16: 5 tiles, the last pair has one
+    (9, (4, 4, 40), 160, 10, [200, 0, 90, 17, 300, 128, 256, 5, 77]),
+])
+def test_two_tiles_per_cta_match_oracle(B, tree, Hq, Hkv, Ls):
+    K, s, N = tree
+    dh = 128
+    Lcap = max(Ls) + N + 5
+    g = torch.Generator(device=DEV).manual_seed(B * 7 + N)
+    q = torch.randn(B, N, Hq, dh, generator=g, device=DEV).bfloat16()
+    kc = torch.randn(B, Lcap, Hkv, dh, generator=g, device=DEV).bfloat16()
+    vc = torch.randn(B, Lcap, Hkv, dh, generator=g, device=DEV).bfloat16()
+    L = torch.tensor(Ls, dtype=torch.int32, device=DEV)
+    t = api.Tree(K, s, N)
+    assert api.attention_tiles_per_cta(t, B, Hq, Hkv, dh, Lcap, torch.bfloat16) == 2
+    assert api.attention_chunks(t, B, Hq, Hkv, dh, Lcap, torch.bfloat16) == 1
+    assert api.attention_launches(t, B, Hq, Hkv, dh, Lcap, torch.bfloat16) == 1
+    scale = 1.0 / math.sqrt(dh)
+    out = api.medusa_tree_attention(q, kc, vc, L, t, scale)
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+    rng = np.random.default_rng(B + N)
+    rows = [(int(rng.integers(B)), int(rng.integers(N)), int(rng.integers(Hq))) for _ in range(160)]
+    # every node of the last rows of each tile pair, on one head of each sequence
+    rows += [(b, i, (b * 7) % Hq) for b in range(B) for i in (0, N // 2 - 1, N // 2, N - 1)]
+    ref = O.tree_attention(q, kc, vc, L, O.tree_plan(K, s, N), scale, rows=rows)
+    got = np.stack([out[b, i, h].double().cpu().numpy() for b, i, h in rows])
+    err = np.abs(got - ref).max()
+    assert err <= ATOL, err
+    assert np.isfinite(out.float().cpu().numpy()).all()
