@@ -254,22 +254,21 @@ TcPlan make_tc_plan(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lc
 }  // namespace
 
 int attention_chunks(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lcap, int dtype) {
-  if (attention_tc_eligible(dtype, dh, Hq, Hkv)) return make_tc_plan(t, B, Hq, Hkv, dh, Lcap).P;
+  if (attention_tc_eligible(dtype, dh, Hq, Hkv)) return attention_tc_shape(B, Hq, Hkv, t->N, Lcap).P;
   return make_plan(t, B, Hq, Hkv, dh, Lcap).chunks;
 }
 
 int attention_tiles_per_cta(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lcap,
                             int dtype) {
   if (!attention_tc_eligible(dtype, dh, Hq, Hkv)) return 1;
-  const int P = make_tc_plan(t, B, Hq, Hkv, dh, Lcap).P;
-  return attention_tc_pair(B, Hq, Hkv, t->N, P) ? 2 : 1;
+  return attention_tc_shape(B, Hq, Hkv, t->N, Lcap).tiles;
 }
 
 int attention_launches(const medusa_tree* t, int B, int Hq, int Hkv, int dh, int Lcap, int dtype) {
   if (B == 0) return 0;
   if (attention_tc_eligible(dtype, dh, Hq, Hkv)) {
-    const int P = make_tc_plan(t, B, Hq, Hkv, dh, Lcap).P;
-    return (P <= 1 || attention_tc_fuse(B, Hq, Hkv, t->N, P)) ? 1 : 2;
+    const TcShape sh = attention_tc_shape(B, Hq, Hkv, t->N, Lcap);
+    return (sh.P <= 1 || sh.fuse) ? 1 : 2;
   }
   return 2;  // SIMT kernel and its combine kernel
 }
@@ -293,14 +292,16 @@ int attention_launch(const AttnArgs& a, cudaStream_t st) {
     if (a.B == 0) return MEDUSA_OK;
     float* po = (float*)((uint8_t*)a.ws + P.off_o);
     float2* pml = (float2*)((uint8_t*)a.ws + P.off_ml);
-    const bool fuse = attention_tc_fuse(a.B, a.Hq, a.Hkv, t->N, P.P);
-    int rc = attention_tc_run(a, P.P, fuse, po, pml, st);
-    if (rc || P.P == 1 || fuse) return rc;
+    const TcShape sh = attention_tc_shape(a.B, a.Hq, a.Hkv, t->N, a.Lcap);
+    if (sh.P > 1 && !sh.fuse && sh.P > P.P)
+      return fail(MEDUSA_ERR_INVALID_ARG, "attention plan exceeds its workspace");
+    int rc = attention_tc_run(a, sh, po, pml, st);
+    if (rc || sh.P == 1 || sh.fuse) return rc;
     const int R = t->N * (a.Hq / a.Hkv);
     const int rows = a.B * t->N * a.Hq;
     cudaError_t e = launch_pdl(tree_attn_combine_kernel<__nv_bfloat16, 128>, dim3((rows + 7) / 8),
                                dim3(256), 0, st, po, pml, a.L, a.B, t->N, a.Hq, a.Hkv, a.Lcap,
-                               P.P, R, (__nv_bfloat16*)a.out);
+                               sh.P, R, (__nv_bfloat16*)a.out);
     if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "tree attention combine launch");
   }

@@ -599,16 +599,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Two query tiles per CTA.  With one key chunk and at least two 128-row query
-// tiles per (sequence, kv-head), a CTA takes tiles 2x and 2x+1 (the second
-// may lie past the last row: computed, never written) and both read every
-// K/V tile it stages.  TMEM: S/P of tile a | S/P of tile b | O of a | O of b.
+// Two query tiles per CTA.  With at least two 128-row query tiles per
+// (sequence, kv-head), a CTA takes tiles 2x and 2x+1 (the second may lie
+// past the last row: computed, never written) and one key chunk, and both
+// tiles read every K/V tile it stages.  With more than one chunk the chunks
+// of a pair form a cluster and merge both tiles' rows in it, as
+// tree_attn_tc_kernel's chunks do.  TMEM: S/P of tile a | S/P of tile b | O of a | O of b.
 // One softmax warpgroup per tile, so each works on its tile while the
 // tensor pipe runs the other tile's MMAs.  S_q(t) reuses the S/P columns of
 // tile q, so it waits for P.V_q(t-1).
 constexpr int kPairKStages = 3, kPairVStages = 2;
 constexpr size_t kPairData = (2 + kPairKStages + kPairVStages) * (size_t)TILE;
 constexpr size_t SMEM_PAIR = 1024 + kPairData + 256;
+static_assert(2 * kOStage + 2 * BM * sizeof(float2) <=
+                  (kPairKStages + kPairVStages) * (size_t)TILE,
+              "both tiles' staged O rows and (max, sum) fit in the K/V rings");
 static_assert(SMEM_PAIR <= 227 * 1024, "shared memory of the two-tile kernel");
 
 // mask_half with the ancestor words of the row's node read from memory (two
@@ -644,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
 
   griddep_wait();  // prefix lengths and the K/V cache may come from the kernel ahead
-  const int qpair = blockIdx.x, bk = blockIdx.z;
+  const int qpair = blockIdx.x, chunk = blockIdx.y, bk = blockIdx.z;
   const int rank = bk / p.Hkv, kvh = bk - rank * p.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* sQ = sm;  // tile a | tile b
@@ -682,11 +687,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int Lb = p.L[b];
   const bool seq_ok = Lb >= 0 && (long long)Lb + p.N <= p.Lcap;
-  const Range rg = chunk_range(p, Lb, 0, seq_ok);
+  const Range rg = chunk_range(p, Lb, chunk, seq_ok);
   const int T = rg.n_pre + rg.n_tree;
   const int qt0 = 2 * qpair;  // tile a; tile b = qt0 + 1
+  const bool b_rows = (qt0 + 1) * BM < p.R;  // tile b has rows to write (uniform in a cluster)
+  // in-cluster merge: staged O rows of tile q at so + q BM OST, (max, sum) at sml + q BM
+  float* so = (float*)(sm + 2 * TILE);
+  float2* sml = (float2*)(sm + 2 * TILE + 2 * kOStage);
 
   if (T == 0) {
+    if (p.fuse) {  // a chunk with no key: (-inf, 0) for every row of both tiles
+      if (threadIdx.x < 2 * BM) sml[threadIdx.x] = make_float2(-INFINITY, 0.f);
+      griddep_launch_dependents();
+      cluster_merge(so, sml, qt0, b, kvh, p.P, p.R, p.G, p.N, p.Hq, p.out);
+      if (b_rows) cluster_merge(so + BM * OST, sml + BM, qt0 + 1, b, kvh, p.P, p.R, p.G, p.N, p.Hq, p.out);
+      return;
+    }
     for (int q = 0; q < 2; ++q) {
       const int grow = (qt0 + q) * BM + (int)threadIdx.x;
       if ((int)threadIdx.x < BM && grow < p.R)
@@ -943,7 +959,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, good);
     }
     const bool bad = bar_red_or(2, 256, !ok || *abort_flag);
-    if (!bad && live) {
+    if (p.fuse) {
+      // stage this chunk's rows for the cluster merge: every MMA has completed
+      // and every K/V load has landed, so the rings are free
+      const bool have = !bad && live && row_ok && m_used != -INFINITY;
+      if (!bad && live) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < DH; c0 += 32) {
+          float a[32];
+          tmem_ld32(tO + (uint32_t)c0, a);
+          if (have) {
+            float4* dst = reinterpret_cast<float4*>(so + ((size_t)q * BM + r) * OST + c0);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(a[4 * e], a[4 * e + 1], a[4 * e + 2], a[4 * e + 3]);
+          }
+        }
+      }
+      sml[q * BM + r] = have ? make_float2(m_used, l) : make_float2(-INFINITY, 0.f);
+    } else if (!bad && live) {
       tc_fence_after();
 #pragma unroll 1
       for (int c0 = 0; c0 < DH; c0 += 32) {
@@ -966,29 +1001,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  if (p.fuse) {
+    cluster_merge(so, sml, qt0, b, kvh, p.P, p.R, p.G, p.N, p.Hq, p.out);
+    if (b_rows) cluster_merge(so + BM * OST, sml + BM, qt0 + 1, b, kvh, p.P, p.R, p.G, p.N, p.Hq, p.out);
+  }
 }
 
 std::atomic<bool> g_smem_attr[64];  // per device: the kernel's shared-memory limit raised
 std::atomic<bool> g_smem_attr_pair[64];
 
-// Clusters of P CTAs of this kernel that can be resident at once on the
-// current device (0 when the query fails), cached per device and P.
-int max_active_clusters(int P) {
-  static std::atomic<int> cache[64][kMaxClusterChunks + 1];
+// Clusters of P CTAs of the one-tile (pair = false) or two-tile kernel that
+// can be resident at once on the current device (0 when the query fails),
+// cached per device, kernel and P.
+int max_active_clusters(bool pair, int P) {
+  static std::atomic<int> cache[2][64][kMaxClusterChunks + 1];
   int dev = 0;
   if (P < 1 || P > kMaxClusterChunks || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     cudaGetLastError();
     return 0;
   }
-  const int v = cache[dev][P].load(std::memory_order_relaxed);
+  const int v = cache[pair][dev][P].load(std::memory_order_relaxed);
   if (v) return v - 1;
-  if (ensure_max_smem(tree_attn_tc_kernel, (int)SMEM, g_smem_attr,
-                      "cudaFuncSetAttribute(tree_attn_tc_kernel)"))
+  const void* fn = pair ? (const void*)tree_attn_tc_pair_kernel : (const void*)tree_attn_tc_kernel;
+  const size_t smem = pair ? SMEM_PAIR : SMEM;
+  if (pair ? ensure_max_smem(tree_attn_tc_pair_kernel, (int)SMEM_PAIR, g_smem_attr_pair,
+                             "cudaFuncSetAttribute(tree_attn_tc_pair_kernel)")
+           : ensure_max_smem(tree_attn_tc_kernel, (int)SMEM, g_smem_attr,
+                             "cudaFuncSetAttribute(tree_attn_tc_kernel)"))
     return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1, P, 1);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = SMEM;
+  cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
@@ -997,11 +1041,11 @@ int max_active_clusters(int P) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, (void*)tree_attn_tc_kernel, &cfg) != cudaSuccess) {
-    cudaGetLastError();  // not an error of the caller's stream: merge with the combine kernel
+  if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
+    cudaGetLastError();  // not an error of the caller's stream: no in-cluster merge
     return 0;
   }
-  cache[dev][P].store(n + 1, std::memory_order_relaxed);
+  cache[pair][dev][P].store(n + 1, std::memory_order_relaxed);
   return n;
 }
 
@@ -1025,30 +1069,60 @@ int attention_tc_chunks(int B, int Hq, int Hkv, int N, int Lcap) {
   return (int)P;
 }
 
-bool attention_tc_pair(int B, int Hq, int Hkv, int N, int P) {
-  if (P != 1 || B <= 0) return false;
+TcShape attention_tc_shape(int B, int Hq, int Hkv, int N, int Lcap) {
+  TcShape sh;
+  sh.P = attention_tc_chunks(B, Hq, Hkv, N, Lcap);
+  sh.tiles = 1;
+  sh.fuse = false;
+  if (B <= 0) return sh;
   const long long R = (long long)N * (Hq / Hkv);
   const long long mtiles = (R + BM - 1) / BM;
-  if (mtiles < 2) return false;
-  // A CTA with two tiles takes about 1.8 times as long per key tile as a CTA
-  // with one (measured on the 8B-GQA and long-context shapes: 2.32-2.35 us
-  // against 1.29-1.34 us), so it pays where it saves enough waves of CTAs.
+  const long long units = (long long)B * Hkv * mtiles;
+  if (sh.P >= 2 && sh.P <= kMaxClusterChunks) {
+    // the chunks of a query tile merge in-cluster when every cluster fits at once
+    const int n = max_active_clusters(false, sh.P);
+    sh.fuse = n > 0 && units <= n;
+  }
+  if (mtiles < 2) return sh;
+  // Cost in (waves of CTAs) x (key tiles per CTA).  A CTA with two query
+  // tiles takes about 1.8 times as long per key tile as a CTA with one
+  // (measured on the 8B-GQA and long-context shapes: 2.32-2.35 us against
+  // 1.29-1.34 us).  Two-tile plans split the keys into P2 chunks only where
+  // the chunks can merge in-cluster.
   const long long sms = num_sms();
-  const long long w1 = ((long long)B * Hkv * mtiles + sms - 1) / sms;
-  const long long w2 = ((long long)B * Hkv * ((mtiles + 1) / 2) + sms - 1) / sms;
-  return 9 * w2 < 5 * w1;
+  const long long T = (Lcap - N + BN - 1) / BN + (N + BN - 1) / BN;
+  const long long cost1 = ((units * sh.P + sms - 1) / sms) * ((T + sh.P - 1) / sh.P);
+  const long long pairs = (long long)B * Hkv * ((mtiles + 1) / 2);
+  const long long max_p = ((long long)(Lcap - N) + 4 * BN - 1) / (4 * BN);  // >= 4 tiles each
+  long long best = cost1 * 10;
+  int bestP = 0;
+  for (int P2 = 1; P2 <= 4; P2 *= 2) {
+    if (P2 > 1 && P2 > max_p) break;
+    long long waves;
+    if (P2 == 1) {
+      waves = (pairs + sms - 1) / sms;
+    } else {
+      const int n = max_active_clusters(true, P2);
+      if (n <= 0) break;
+      waves = (pairs + n - 1) / n;
+    }
+    const long long cost2 = 18 * waves * ((T + P2 - 1) / P2);
+    if (cost2 < best) {
+      best = cost2;
+      bestP = P2;
+    }
+  }
+  if (bestP > 0) {
+    sh.P = bestP;
+    sh.tiles = 2;
+    sh.fuse = bestP > 1;
+  }
+  return sh;
 }
 
-bool attention_tc_fuse(int B, int Hq, int Hkv, int N, int P) {
-  if (P < 2 || P > kMaxClusterChunks || B <= 0) return false;
-  const long long R = (long long)N * (Hq / Hkv);
-  const long long units = (long long)B * Hkv * ((R + BM - 1) / BM);
-  const int n = max_active_clusters(P);
-  return n > 0 && units <= n;
-}
-
-int attention_tc_run(const AttnArgs& a, int P, bool fuse, float* po, float2* pml,
+int attention_tc_run(const AttnArgs& a, const TcShape& sh, float* po, float2* pml,
                      cudaStream_t st) {
+  const int P = sh.P;
   const medusa_tree* t = a.tree;
   const int G = a.Hq / a.Hkv;
   const int R = t->N * G;
@@ -1086,24 +1160,20 @@ int attention_tc_run(const AttnArgs& a, int P, bool fuse, float* po, float2* pml
   p.R = R;
   p.P = P;
   p.mtiles = mtiles;
-  p.fuse = (fuse && P >= 2 && P <= kMaxClusterChunks) ? 1 : 0;
+  p.fuse = (sh.fuse && P >= 2 && P <= kMaxClusterChunks) ? 1 : 0;
   p.qscale = a.scale * 1.4426950408889634f;
   p.out = (__nv_bfloat16*)a.out;
   p.po = po;
   p.pml = pml;
   cudaError_t e;
-  if (attention_tc_pair(a.B, a.Hq, a.Hkv, t->N, P)) {
-    // two query tiles per CTA (one key chunk)
+  const bool pair = sh.tiles == 2;
+  if (pair && P > 1 && !p.fuse) return fail(MEDUSA_ERR_UNSUPPORTED, "two-tile plan without merge");
+  if (pair) {
     rc = ensure_max_smem(tree_attn_tc_pair_kernel, (int)SMEM_PAIR, g_smem_attr_pair,
                          "cudaFuncSetAttribute(tree_attn_tc_pair_kernel)");
     if (rc) return rc;
-    p.fuse = 0;
-    e = launch_pdl(tree_attn_tc_pair_kernel, dim3((mtiles + 1) / 2, 1, a.B * a.Hkv),
-                   dim3(kThreads), SMEM_PAIR, st, mQ, mK, mV, p);
-    if (e == cudaSuccess) e = cudaGetLastError();
-    return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "tree_attn_tc_pair_kernel launch");
   }
-  dim3 grid(mtiles, P, a.B * a.Hkv);
+  dim3 grid(pair ? (mtiles + 1) / 2 : mtiles, P, a.B * a.Hkv);
   if (p.fuse) {
     // the P chunks of a query tile (grid y) are one cluster
     cudaLaunchConfig_t cfg = {};
@@ -1120,7 +1190,14 @@ int attention_tc_run(const AttnArgs& a, int P, bool fuse, float* po, float2* pml
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    e = cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel, mQ, mK, mV, p);
+    if (pair) {
+      cfg.dynamicSmemBytes = SMEM_PAIR;
+      e = cudaLaunchKernelEx(&cfg, tree_attn_tc_pair_kernel, mQ, mK, mV, p);
+    } else {
+      e = cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel, mQ, mK, mV, p);
+    }
+  } else if (pair) {
+    e = launch_pdl(tree_attn_tc_pair_kernel, grid, dim3(kThreads), SMEM_PAIR, st, mQ, mK, mV, p);
   } else {
     e = launch_pdl(tree_attn_tc_kernel, grid, dim3(kThreads), SMEM, st, mQ, mK, mV, p);
   }

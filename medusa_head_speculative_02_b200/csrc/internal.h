@@ -138,12 +138,18 @@ int attention_tiles_per_cta(const medusa_tree* t, int B, int Hq, int Hkv, int dh
 // tcgen05 path (bf16, dh = 128, GQA group dividing 128)
 bool attention_tc_eligible(int dtype, int dh, int Hq, int Hkv);
 int attention_tc_chunks(int B, int Hq, int Hkv, int N, int Lcap);
-// true when the P key chunks of every query tile run as one thread-block
-// cluster, all clusters resident at once, and merge inside the kernel
-bool attention_tc_fuse(int B, int Hq, int Hkv, int N, int P);
-// true when each CTA takes two query tiles of a (sequence, kv-head) (one key chunk)
-bool attention_tc_pair(int B, int Hq, int Hkv, int N, int P);
-int attention_tc_run(const AttnArgs& a, int P, bool fuse, float* po, float2* pml,
+// Launch shape of the tensor-core attention: P key chunks per query tile,
+// `tiles` (1 or 2) 128-row query tiles per CTA, and whether the chunks of a
+// query tile run as one thread-block cluster and merge inside the kernel
+// (else, with P > 1, the combine kernel merges them; two-tile shapes with
+// P > 1 always merge in-cluster).
+struct TcShape {
+  int P;
+  int tiles;
+  bool fuse;
+};
+TcShape attention_tc_shape(int B, int Hq, int Hkv, int N, int Lcap);
+int attention_tc_run(const AttnArgs& a, const TcShape& sh, float* po, float2* pml,
                      cudaStream_t st);
 
 // ---------------------------------------------------------------- acceptance

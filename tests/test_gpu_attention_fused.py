@@ -67,14 +67,16 @@ def test_fused_merge_is_repeatable_and_leaves_no_state():
 
 
 # ---------------------------------------------------------------- two query tiles per CTA
-@pytest.mark.parametrize("B,tree,Hq,Hkv,Ls", [
+@pytest.mark.parametrize("B,tree,Hq,Hkv,Ls,chunks", [
     # GQA 4: 4 query tiles per (sequence, kv-head), 512 single-tile CTAs
     (16, (5, 8, 128), 32, 8, [50, 400, 120, 333, 7, 260, 199, 380, 0, 64, 128, 129, 255, 256,
-                              300, 1]),
+                              300, 1], 1),
     # GQA 16: 5 tiles, the last pair has one
-    (9, (4, 4, 40), 160, 10, [200, 0, 90, 17, 300, 128, 256, 5, 77]),
+    (9, (4, 4, 40), 160, 10, [200, 0, 90, 17, 300, 128, 256, 5, 77], 1),
+    # 256 tree nodes, 52 heads (2 tiles): keys split in 2 chunks, merged in-cluster
+    (4, (5, 3, 256), 52, 52, [2000, 1500, 700, 1999], 2),
 ])
-def test_two_tiles_per_cta_match_oracle(B, tree, Hq, Hkv, Ls):
+def test_two_tiles_per_cta_match_oracle(B, tree, Hq, Hkv, Ls, chunks):
     K, s, N = tree
     dh = 128
     Lcap = max(Ls) + N + 5
@@ -85,7 +87,7 @@ def test_two_tiles_per_cta_match_oracle(B, tree, Hq, Hkv, Ls):
     L = torch.tensor(Ls, dtype=torch.int32, device=DEV)
     t = api.Tree(K, s, N)
     assert api.attention_tiles_per_cta(t, B, Hq, Hkv, dh, Lcap, torch.bfloat16) == 2
-    assert api.attention_chunks(t, B, Hq, Hkv, dh, Lcap, torch.bfloat16) == 1
+    assert api.attention_chunks(t, B, Hq, Hkv, dh, Lcap, torch.bfloat16) == chunks
     assert api.attention_launches(t, B, Hq, Hkv, dh, Lcap, torch.bfloat16) == 1
     scale = 1.0 / math.sqrt(dh)
     out = api.medusa_tree_attention(q, kc, vc, L, t, scale)
