@@ -191,7 +191,9 @@ int medusa_build_tree(const medusa_tree_t* tree, const int32_t* root_tok,
  * violates it are written as zeros and the status word is left untouched),
  * Hq % Hkv == 0, dh in {64, 128}, scale finite and > 0 (normally
  * 1/sqrt(dh)).  bf16 with dh = 128 and (Hq/Hkv) dividing 128 runs on the
- * tcgen05 tensor-core kernel; other shapes on a SIMT kernel.
+ * tcgen05 tensor-core kernels (one or two 128-row query tiles per CTA, keys
+ * split into chunks where that fills the device; the choice is reported by
+ * the introspection calls below); other shapes on a SIMT kernel.
  * ------------------------------------------------------------------------ */
 size_t medusa_tree_attention_workspace_size(const medusa_tree_t* tree, int B,
                                             int Hq, int Hkv, int dh, int Lcap);
