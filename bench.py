@@ -146,8 +146,9 @@ def measured_peaks() -> dict:
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         d = json.load(open(path))
-        return {"hbm_gbs": d.get("hbm_gbs", 6650.0), "src": "measured"}
-    return {"hbm_gbs": 6650.0, "src": "fallback"}
+        return {"hbm_gbs": d.get("hbm_gbs", 6650.0), "bf16_tflops": d.get("bf16_tflops", 1590.0),
+                "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "src": "fallback"}
 
 
 # ---------------------------------------------------------------------------- oracle sampler
@@ -449,6 +450,7 @@ def run_ours(args, cfg, world, rank, local):
     sample_bytes = cfg.B * cfg.V * (4 if cfg.dtype == "f32" else 2)
     hb = st.heads_bytes()
     ab = st.attention_bytes()
+    af = st.attention_flops()
     heads_gbs = hb / (heads_ms / 1000.0) / 1e9
     attn_gbs = ab / (attn_ms / 1000.0) / 1e9
     traffic = None
@@ -486,6 +488,10 @@ def run_ours(args, cfg, world, rank, local):
                 "kernels": {"tree_attention": {"achieved": attn_gbs, "unit": "GB/s",
                                                "frac": attn_gbs / peaks["hbm_gbs"],
                                                "algorithmic_bytes": ab, "avg_ms": attn_ms,
+                                               "tflops": af / (attn_ms / 1000.0) / 1e12,
+                                               "tensor_frac": af / (attn_ms / 1000.0) / 1e12
+                                               / peaks["bf16_tflops"],
+                                               "algorithmic_flops": af,
                                                "key_chunks": attn_chunks,
                                                "query_tiles_per_cta": attn_tiles,
                                                "launches": attn_launches},

@@ -109,6 +109,13 @@ class VerifyStep:
         e = 4 if c.dtype == "f32" else 2
         return e * (c.K * c.d * c.d + c.K * c.d + c.K * c.V * c.d + c.B * c.d) + 8 * c.B * c.K * c.s
 
+    def attention_flops(self) -> int:
+        """Tensor-core work of the attention call: S = Q K^T and O = P V over
+        every key of a sequence's prefix and tree slots, per query row."""
+        c = self.cfg
+        Lsum = int(self.x["prefix_len"].sum().item())
+        return 4 * c.Hq * c.N * (Lsum + c.B * c.N) * c.dh
+
     def attention_bytes(self) -> int:
         """K/V actually read (prefix + tree slots) + Q + O."""
         c = self.cfg
