@@ -12,7 +12,10 @@
 // pair is an independent CTA producing unnormalised partial outputs with
 // their running max / sum in base 2, and a combine kernel merges the chunks
 // of every query row.  All query rows of a kv-head (tree nodes x the GQA
-// group) share each staged K/V tile.
+// group) share each staged K/V tile.  This SIMT kernel serves fp32 and
+// dh = 64; attention_launch sends bf16 with dh = 128 to the tensor-core
+// kernels of attention_tc.cu, whose launch shape (query tiles per CTA, key
+// chunks, in-cluster merge) attention_tc_shape chooses.
 #include "common.cuh"
 #include "internal.h"
 
