@@ -102,3 +102,19 @@ def test_two_tiles_per_cta_match_oracle(B, tree, Hq, Hkv, Ls, chunks):
     err = np.abs(got - ref).max()
     assert err <= ATOL, err
     assert np.isfinite(out.float().cpu().numpy()).all()
+
+
+def test_plan_queries_reject_bad_shapes():
+    t = api.Tree(5, 10, 64)
+    for fn in (api.attention_chunks, api.attention_launches, api.attention_tiles_per_cta):
+        with pytest.raises(RuntimeError):
+            fn(t, 1, 6, 4, 128, 4096, torch.bfloat16)    # Hq not a multiple of Hkv
+        with pytest.raises(RuntimeError):
+            fn(t, -1, 4, 4, 128, 4096, torch.bfloat16)   # negative batch
+        with pytest.raises(RuntimeError):
+            fn(t, 1, 4, 4, 128, 32, torch.bfloat16)      # cache shorter than the tree
+    # no sequences: no launch
+    assert api.attention_launches(t, 0, 4, 4, 128, 4096, torch.bfloat16) == 0
+    # the tiny fp32 shape runs on the SIMT kernel and its combine kernel, one tile per CTA
+    assert api.attention_launches(t, 1, 4, 4, 64, 4096, torch.float32) == 2
+    assert api.attention_tiles_per_cta(t, 1, 4, 4, 64, 4096, torch.float32) == 1

@@ -99,3 +99,27 @@ def test_validation_before_any_launch():
     st = C.c_int()
     assert lib.medusa_device_status(None, 0) == L.ERR_INVALID_ARG
     assert lib.medusa_heads_workspace_size(0, 64, 10, 2, 1, L.BF16) == 0
+
+
+def test_shard_merge_and_attention_plan_queries_validate_first():
+    """The shard merge and the attention plan queries reject bad arguments
+    before any CUDA call."""
+    lib = L.lib()
+    p = C.c_void_p(256)
+    # G < 1, c < 1, s out of range, shard stride below R * c, NULL outputs
+    assert lib.medusa_topk_merge(p, p, 40, None, 0, 4, 10, 10, p, p, None) == L.ERR_INVALID_ARG
+    assert lib.medusa_topk_merge(p, p, 40, None, 2, 4, 0, 10, p, p, None) == L.ERR_INVALID_ARG
+    assert lib.medusa_topk_merge(p, p, 40, None, 2, 4, 10, 0, p, p, None) == L.ERR_INVALID_ARG
+    assert lib.medusa_topk_merge(p, p, 40, None, 2, 4, 10, 17, p, p, None) == L.ERR_INVALID_ARG
+    assert lib.medusa_topk_merge(p, p, 39, None, 2, 4, 10, 10, p, p, None) == L.ERR_INVALID_ARG
+    assert lib.medusa_topk_merge(p, p, 40, None, 2, 4, 10, 10, None, p, None) == \
+        L.ERR_INVALID_ARG
+    assert lib.medusa_topk_merge(None, p, 40, None, 2, 4, 10, 10, p, p, None) == \
+        L.ERR_INVALID_ARG
+    # no rows: nothing to do, accepted without touching the pointers
+    assert lib.medusa_topk_merge(None, None, 0, None, 2, 0, 10, 10, None, None, None) == L.OK
+    # plan queries reject a NULL tree (the other checks need a tree, whose
+    # plan lives on the device)
+    for fn in (lib.medusa_tree_attention_chunks, lib.medusa_tree_attention_launches,
+               lib.medusa_tree_attention_tiles_per_cta):
+        assert fn(None, 1, 4, 4, 128, 4096, L.BF16) == L.ERR_INVALID_ARG
