@@ -188,7 +188,10 @@ int medusa_build_tree(const medusa_tree_t* tree, const int32_t* root_tok,
  * h / (Hq/Hkv).
  * q [B][N][Hq][dh]; k_cache, v_cache [B][Lcap][Hkv][dh]; out [B][N][Hq][dh].
  * Requires L_b + N <= Lcap (checked on the device: rows of a sequence that
- * violates it are written as zeros and the status word is left untouched),
+ * violates it are written as zeros and the status word is left untouched).
+ * Slots 0..L_b+N-1 of sequence b must hold finite values; slots L_b+N and
+ * beyond (unused capacity) may hold anything, NaN and Inf included: they get
+ * weight exactly 0 and never reach the output.  Further requirements:
  * Hq % Hkv == 0, dh in {64, 128}, scale finite and > 0 (normally
  * 1/sqrt(dh)).  bf16 with dh = 128 and (Hq/Hkv) dividing 128 runs on the
  * tcgen05 tensor-core kernels (one or two 128-row query tiles per CTA, keys

@@ -24,8 +24,13 @@
 //                   the O row is then rescaled in TMEM once the previous P.V
 //                   is done), P = 2^(scale*s - m) with packed fp32x2
 //                   arithmetic, one pair in four of the exponentials on the
-//                   FMA pipe (polynomial) and the rest on MUFU, written as
-//                   bf16 pairs over the S columns just read
+//                   FMA pipe (polynomial) and the rest on MUFU (all on MUFU
+//                   in a key half with masked keys, so those weigh exactly
+//                   0), written as bf16 pairs over the S columns just read;
+//                   on a tile that reaches past slot L_b + N the softmax
+//                   warps first zero those V rows in shared memory (cache
+//                   slots the caller need not have written: NaN or Inf
+//                   there would otherwise reach O through 0 * NaN)
 //   O += P V        tcgen05.mma (M 128, N 128, K 128): A = P from TMEM, V
 //                   the MN-major smem operand
 // TMEM (512 columns): three S/P buffers and O, 128 columns each.  Warp 0
@@ -154,6 +159,65 @@ __device__ __forceinline__ void mask_half(float (&v)[64], int j, int hf, const R
       const bool vis = c < nvalid && ((word >> (c & 31)) & 1u);
       v[c] = vis ? v[c] : -INFINITY;
     }
+  }
+}
+
+// P = 2^(qscale * s - m) for the 64 scores of one key half, packed as bf16
+// pairs (pk[c] holds keys 2c, 2c+1); returns their fp32 sum.  kMasked: the
+// half holds masked (-inf) scores, so every exponential goes to MUFU ex2,
+// which gives exactly 0 there; otherwise one pair in four is taken on the
+// FMA pipe (polynomial), which would give 2^-126 for -inf.
+template <bool kMasked>
+__device__ __forceinline__ float exp_pack64(const float (&v)[64], unsigned long long q2,
+                                            unsigned long long m2, uint32_t (&pk)[32]) {
+  unsigned long long sum2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int c2 = 0; c2 < 32; ++c2) {
+    float x0, x1, e0, e1;
+    f2_unpack(f2_fma(f2_pack(v[2 * c2], v[2 * c2 + 1]), q2, m2), x0, x1);
+    if (!kMasked && (c2 & 3) == 3) {
+      exp2_fma2(x0, x1, e0, e1);
+    } else {
+      e0 = ex2_approx(x0);
+      e1 = ex2_approx(x1);
+    }
+    sum2[c2 & 3] = f2_add(sum2[c2 & 3], f2_pack(e0, e1));
+    const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
+    pk[c2] = *reinterpret_cast<const uint32_t*>(&h2);
+  }
+  float a0, a1, b0, b1, c0f, c1f, d0, d1;
+  f2_unpack(sum2[0], a0, a1);
+  f2_unpack(sum2[1], b0, b1);
+  f2_unpack(sum2[2], c0f, c1f);
+  f2_unpack(sum2[3], d0, d1);
+  return ((a0 + a1) + (b0 + b1)) + ((c0f + c1f) + (d0 + d1));
+}
+
+// True when the 64-key half hf of key tile j has masked columns: a tree
+// tile, or the prefix tile that ends the chunk inside this half.
+__device__ __forceinline__ bool half_masked(int j, int hf, const Range& rg) {
+  return j >= rg.n_pre || rg.k_hi - (rg.k_lo + j * BN + hf * 64) < 64;
+}
+
+// First cache slot of key tile j (prefix tiles from the chunk start, then the
+// tree tiles from slot L_b).
+__device__ __forceinline__ int tile_key0(int j, int Lb, const Range& rg) {
+  return j < rg.n_pre ? rg.k_lo + j * BN : Lb + (j - rg.n_pre) * BN;
+}
+
+// Zeroes rows [row0, BN) of a staged 128-key V tile (both 64-column halves;
+// the 128-byte swizzle permutes 16-byte pieces within a row, so a whole row
+// stays at bytes [128 row, 128 row + 128) of each half).  Those rows hold
+// cache slots >= L_b + N, which the caller never has to write: their
+// attention weight is exactly 0, and zero rows keep 0 * (NaN or Inf) out of
+// the P.V product.  nthr threads, index i; the caller orders the stores
+// before the tensor core's reads (proxy fence, then barrier).
+__device__ __forceinline__ void zero_v_rows(uint8_t* tile, int row0, int i, int nthr) {
+  const int n = (BN - row0) * 16;  // 16-byte pieces: 8 per row and half
+  for (int e = i; e < n; e += nthr) {
+    const int row = row0 + (e >> 4), pc = e & 15;
+    *reinterpret_cast<uint4*>(tile + (pc >> 3) * HALF + row * 128 + (pc & 7) * 16) =
+        make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
@@ -443,6 +507,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tS = tmem + lane_base + (uint32_t)(bf * 128 + hf * 64);
       const bool good = mbar_wait(&s_full[bf], (uint32_t)(t / 3) & 1u, abort_flag);
       err = err || !__all_sync(0xffffffffu, good);
+      // V rows of cache slots >= L_b + N in this tile (the tree tiles and the
+      // prefix tile that ends the sequence): zeroed by the 256 softmax
+      // threads once the tile has landed, before P(t) is released to P.V(t)
+      const int zrow = Lb + p.N - tile_key0(t, Lb, rg);
+      if (zrow < BN && !err) {
+        const int vs = t % kStages;
+        const bool vg = mbar_wait(&v_full[vs], (uint32_t)(t / kStages) & 1u, abort_flag);
+        if (__all_sync(0xffffffffu, vg)) {
+          zero_v_rows(sV + vs * TILE, zrow, (int)threadIdx.x - 64, 256);
+          fence_proxy_async_smem();
+        } else {
+          err = true;
+        }
+      }
       float v[64];
       float tmax = -INFINITY;
       // Both halves of a row use max(round_up(max_0), round_up(max_1)): the
@@ -500,34 +578,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // has m = -inf and only -inf scores, whose exponentials are zeroed)
       const float moff = (m_used == -INFINITY) ? 0.f : m_used;
       const unsigned long long m2 = f2_pack(-moff, -moff);
-      unsigned long long sum2[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pk[32];
-#pragma unroll
-      for (int c2 = 0; c2 < 32; ++c2) {
-        float x0, x1, e0, e1;
-        f2_unpack(f2_fma(f2_pack(v[2 * c2], v[2 * c2 + 1]), q2, m2), x0, x1);
-        if ((c2 & 3) == 3) {
-          // a masked key gives 2^-126 here rather than 0: negligible next
-          // to the row sum (>= 1 once a key is visible), and wiped by the
-          // zero rescale while the row has seen no visible key
-          exp2_fma2(x0, x1, e0, e1);
-        } else {
-          e0 = ex2_approx(x0);
-          e1 = ex2_approx(x1);
-        }
-        sum2[c2 & 3] = f2_add(sum2[c2 & 3], f2_pack(e0, e1));
-        const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
-        pk[c2] = *reinterpret_cast<const uint32_t*>(&h2);
-      }
+      // masked keys get exactly 0 (all-MUFU exponentials on masked halves)
+      l += half_masked(t, hf, rg) ? exp_pack64<true>(v, q2, m2, pk)
+                                  : exp_pack64<false>(v, q2, m2, pk);
       tmem_st32(tS, pk);  // P over the S columns just read
-      {
-        float a0, a1, b0, b1, c0f, c1f, d0, d1;
-        f2_unpack(sum2[0], a0, a1);
-        f2_unpack(sum2[1], b0, b1);
-        f2_unpack(sum2[2], c0f, c1f);
-        f2_unpack(sum2[3], d0, d1);
-        l += ((a0 + a1) + (b0 + b1)) + ((c0f + c1f) + (d0 + d1));
-      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[bf]);
@@ -908,6 +963,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false;
         break;
       }
+      // V rows of cache slots >= L_b + N in this tile: zeroed by tile a's
+      // warpgroup before P_a(t) is released; the MMA thread issues P.V_b(t)
+      // after P.V_a(t), so both products read the zeroed rows
+      const int zrow = Lb + p.N - tile_key0(t, Lb, rg);
+      if (q == 0 && zrow < BN) {
+        const int vs = t % kPairVStages;
+        const bool vg = mbar_wait(&v_full[vs], (uint32_t)(t / kPairVStages) & 1u, abort_flag);
+        if (!__all_sync(0xffffffffu, vg)) {
+          ok = false;
+          break;
+        }
+        zero_v_rows(sV + vs * TILE, zrow, (int)threadIdx.x - 64, 128);
+        fence_proxy_async_smem();
+      }
       if (live) {
 #pragma unroll 1
         for (int hf = 0; hf < 2 && ok; ++hf) {
@@ -923,29 +992,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           // yet has m = -inf and only -inf scores, whose exponentials are zeroed)
           const float moff = (m_used == -INFINITY) ? 0.f : m_used;
           const unsigned long long m2 = f2_pack(-moff, -moff);
-          unsigned long long sum2[4] = {0ull, 0ull, 0ull, 0ull};
           uint32_t pk[32];
-#pragma unroll
-          for (int c2 = 0; c2 < 32; ++c2) {
-            float x0, x1, e0, e1;
-            f2_unpack(f2_fma(f2_pack(v[2 * c2], v[2 * c2 + 1]), q2, m2), x0, x1);
-            if ((c2 & 3) == 3) {
-              exp2_fma2(x0, x1, e0, e1);
-            } else {
-              e0 = ex2_approx(x0);
-              e1 = ex2_approx(x1);
-            }
-            sum2[c2 & 3] = f2_add(sum2[c2 & 3], f2_pack(e0, e1));
-            const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
-            pk[c2] = *reinterpret_cast<const uint32_t*>(&h2);
-          }
+          // masked keys get exactly 0 (all-MUFU exponentials on masked halves)
+          l += half_masked(t, hf, rg) ? exp_pack64<true>(v, q2, m2, pk)
+                                      : exp_pack64<false>(v, q2, m2, pk);
           tmem_st32(tS + (uint32_t)(hf * 64), pk);  // P over the S columns just read
-          float a0, a1, b0, b1, c0f, c1f, d0, d1;
-          f2_unpack(sum2[0], a0, a1);
-          f2_unpack(sum2[1], b0, b1);
-          f2_unpack(sum2[2], c0f, c1f);
-          f2_unpack(sum2[3], d0, d1);
-          l += ((a0 + a1) + (b0 + b1)) + ((c0f + c1f) + (d0 + d1));
         }
         if (!ok) break;
       }

@@ -10,12 +10,12 @@ import numpy as np
 import pytest
 import torch
 
+from attn_check import assert_attention_close
 from oracle import medusa_oracle as O
 from medusa_head_speculative_02_b200 import api
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
-ATOL = 2e-2
 
 
 @pytest.mark.parametrize("B,tree,Hq,Hkv,Ls", [
@@ -43,8 +43,7 @@ def test_fused_chunk_merge_matches_oracle(B, tree, Hq, Hkv, Ls):
     out = api.medusa_tree_attention(q, kc, vc, L, t, scale)
     torch.cuda.synchronize()
     ref = O.tree_attention(q, kc, vc, L, O.tree_plan(K, s, N), scale)
-    err = np.abs(out.double().cpu().numpy() - ref).max()
-    assert err <= ATOL, err
+    assert_attention_close(out.double().cpu().numpy(), ref, what=f"B={B} Hq={Hq} L={Ls} P={P}")
     assert api.device_status() == 0
 
 
@@ -99,8 +98,7 @@ def test_two_tiles_per_cta_match_oracle(B, tree, Hq, Hkv, Ls, chunks):
     rows += [(b, i, (b * 7) % Hq) for b in range(B) for i in (0, N // 2 - 1, N // 2, N - 1)]
     ref = O.tree_attention(q, kc, vc, L, O.tree_plan(K, s, N), scale, rows=rows)
     got = np.stack([out[b, i, h].double().cpu().numpy() for b, i, h in rows])
-    err = np.abs(got - ref).max()
-    assert err <= ATOL, err
+    assert_attention_close(got, ref, what=f"B={B} Hq={Hq} Hkv={Hkv} N={N}")
     assert np.isfinite(out.float().cpu().numpy()).all()
 
 

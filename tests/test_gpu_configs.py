@@ -12,6 +12,7 @@ import numpy as np
 import pytest
 import torch
 
+from attn_check import assert_attention_close
 from oracle import medusa_oracle as O
 from medusa_head_speculative_02_b200 import api
 from medusa_head_speculative_02_b200.step import VerifyStep
@@ -89,8 +90,27 @@ def test_attention_full_size_sampled(step):
     ref = O.tree_attention(x["q"], x["k_cache"], x["v_cache"], x["prefix_len"], plan,
                            1.0 / math.sqrt(cfg.dh), rows=rows)
     got = np.stack([out[b, i, h].double().cpu().numpy() for (b, i, h) in rows])
-    tol = 1e-4 if cfg.dtype == "f32" else ATOL
-    assert np.abs(got - ref).max() <= tol
+    assert_attention_close(got, ref, bf16=cfg.dtype == "bf16", what=f"{cfg.name} sampled rows")
+
+
+def test_attention_full_size_whole_kv_head(step):
+    """Every output row of one (sequence, kv-head): all tree nodes x the GQA
+    group, so every query tile of the pair, every key chunk and every tree
+    tile is compared, on the sequence with the longest prefix."""
+    cfg, x = step.cfg, step.x
+    step.attention()
+    torch.cuda.synchronize()
+    out = step.attn_out
+    plan = O.tree_plan(cfg.K, cfg.s, cfg.N)
+    b = int(torch.argmax(x["prefix_len"]).item())
+    kvh = cfg.Hkv - 1
+    G = cfg.Hq // cfg.Hkv
+    rows = [(b, i, kvh * G + g) for i in range(cfg.N) for g in range(G)]
+    ref = O.tree_attention(x["q"], x["k_cache"], x["v_cache"], x["prefix_len"], plan,
+                           1.0 / math.sqrt(cfg.dh), rows=rows)
+    got = out[b, :, kvh * G:(kvh + 1) * G].double().cpu().numpy().reshape(-1, cfg.dh)
+    assert_attention_close(got, ref, bf16=cfg.dtype == "bf16",
+                           what=f"{cfg.name} sequence {b} kv-head {kvh}, {len(rows)} rows")
 
 
 def _accept_inputs(cfg, tree_parent):

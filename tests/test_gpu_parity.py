@@ -8,6 +8,7 @@ import numpy as np
 import pytest
 import torch
 
+from attn_check import assert_attention_close
 from oracle import medusa_oracle as O
 from medusa_head_speculative_02_b200 import api
 from medusa_head_speculative_02_b200.synthetic import (CONFIGS, MedusaConfig, gen_inputs,
@@ -148,8 +149,8 @@ def test_tree_attention_small(B, tree, Hq, Hkv, dh, Ls, dtype):
     scale = 1.0 / math.sqrt(dh)
     out = api.medusa_tree_attention(q, kc, vc, L, t, scale)
     ref = O.tree_attention(q, kc, vc, L, plan, scale)
-    err = np.abs(out.double().cpu().numpy() - ref).max()
-    assert err <= (1e-4 if dtype == torch.float32 else ATOL), err
+    assert_attention_close(out.double().cpu().numpy(), ref, bf16=dtype == torch.bfloat16,
+                           what=f"B={B} tree={tree} Hq={Hq} Hkv={Hkv} dh={dh} L={Ls}")
 
 
 def test_tree_attention_chain_equals_causal_sdpa():
@@ -168,7 +169,7 @@ def test_tree_attention_chain_equals_causal_sdpa():
     ref = torch.nn.functional.scaled_dot_product_attention(
         qf, kc.double().cpu().permute(0, 2, 1, 3), vc.double().cpu().permute(0, 2, 1, 3),
         is_causal=True, scale=1 / math.sqrt(dh))[:, :, L:].permute(0, 2, 1, 3)
-    assert (out.double().cpu() - ref).abs().max().item() <= ATOL
+    assert_attention_close(out.double().cpu().numpy(), ref.numpy(), what="chain tree")
 
 
 def test_tree_attention_rejects_overflowing_sequence_rows():
@@ -179,7 +180,7 @@ def test_tree_attention_rejects_overflowing_sequence_rows():
     out = api.medusa_tree_attention(q, kc, vc, L, t, 0.1)
     assert out[1].abs().max().item() == 0.0
     ref = O.tree_attention(q[:1], kc[:1], vc[:1], L[:1], O.tree_plan(K, s, N), 0.1)
-    assert np.abs(out[:1].double().cpu().numpy() - ref).max() <= ATOL
+    assert_attention_close(out[:1].double().cpu().numpy(), ref, what="valid sequence")
 
 
 # ---------------------------------------------------------------------------- acceptance
