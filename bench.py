@@ -8,6 +8,13 @@ One process per GPU (torchrun for N > 1).  Every rank runs its own replica
 of the step on its own sequences (data parallel, no collective on the data
 path: weak scaling).  Rank 0 prints one JSON line.  `--impl reference` times
 the plain fp64 CPU oracle on sampled slices of the same workload.
+
+The timed region is K verify steps back to back, with no event between
+them.  The per-kernel figures (heads, tree attention, acceptance) come from
+separate loops of back-to-back calls of each entry point after it
+(medusa_head_speculative_02_b200.kernel_bench); the dominant kernel of the
+step is the `roofline` object.  The other workloads' step rates and kernel
+figures follow under `configs`.
 """
 from __future__ import annotations
 
@@ -26,11 +33,14 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from medusa_head_speculative_02_b200.synthetic import CONFIGS, gen_inputs  # noqa: E402
+from medusa_head_speculative_02_b200.synthetic import CONFIG_ORDER, CONFIGS, gen_inputs  # noqa: E402
 
-DEFAULT_CONFIG = "7b_b1"
+# the largest workload that fits one GPU: B = 4 sequences of 32K-token prefixes,
+# 256-node trees, d = 6656
+DEFAULT_CONFIG = "longctx_b4"
 METRIC = "verify steps/s"
-EVENT_EVERY = 8  # timed steps per step whose heads / attention calls are bracketed by events
+KERNEL_CALLS = 50   # back-to-back calls per entry point for the per-kernel figures
+EXTRA_STEPS = 50    # timed steps of each of the other workloads
 DECODE_STEPS = 128  # chained steps of the decode-loop measurement
 SAMPLE_REPS = 50    # timed calls of the sampled-next-token measurement
 SHARD_REPS = 50     # timed calls per shard count of the vocabulary-sharded heads
@@ -142,15 +152,6 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
-def measured_peaks() -> dict:
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(path):
-        d = json.load(open(path))
-        return {"hbm_gbs": d.get("hbm_gbs", 6650.0), "bf16_tflops": d.get("bf16_tflops", 1590.0),
-                "src": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "src": "fallback"}
-
-
 # ---------------------------------------------------------------------------- oracle sampler
 class OracleSampler:
     """Times the fp64 CPU oracle on bounded slices of one verify step and
@@ -236,6 +237,56 @@ class OracleSampler:
                 "; each op's mean slice time scaled by full/slice units and summed")
 
 
+def oracle_full_step_seconds(cfg) -> float:
+    """Wall time of one whole verify step of the oracle on the host (every
+    head logit, every attention row, both acceptance rules where the workload
+    has them, the compaction), inputs generated beforehand."""
+    from oracle import medusa_oracle as O
+    from medusa_head_speculative_02_b200.synthetic import plant_verify_logits
+    x = gen_inputs(cfg, "cpu", seed=0)
+    t0 = time.perf_counter()
+    plan = O.tree_plan(cfg.K, cfg.s, cfg.N)
+    logits = O.heads_forward(x["h"], x["W1"], x["b1"], x["W2"])
+    tk = O.topk(logits, cfg.s)
+    tok, _ = O.build_tree(plan, x["root_tok"], tk, x["prefix_len"])
+    O.tree_attention(x["q"], x["k_cache"], x["v_cache"], x["prefix_len"], plan,
+                     1.0 / np.sqrt(cfg.dh))
+    t1 = time.perf_counter()
+    vlog = plant_verify_logits(cfg, plan["parent"], tok, "cpu", 0)   # input, not timed
+    t2 = time.perf_counter()
+    if cfg.accept in ("greedy", "both"):
+        alen, anodes, _ = O.accept_greedy(vlog, tok, plan)
+    if cfg.accept in ("typical", "both"):
+        alen, anodes, _, _ = O.accept_typical(vlog, tok, plan, cfg.temperature, cfg.eps,
+                                              cfg.delta)
+    O.kv_compact(x["k_cache"], x["v_cache"], x["prefix_len"], alen, anodes)
+    return (t1 - t0) + (time.perf_counter() - t2)
+
+
+FULL_STEP_WORKLOADS = ("tiny_f32", "7b_b1")
+
+
+def cpu_baseline(S, seconds: float) -> dict:
+    """The oracle on this host: the headline workload extrapolated from timed
+    slices, and whole steps of the two smallest workloads measured in full."""
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        S.step()
+    est = S.estimate_step_seconds()
+    full = {}
+    for name in FULL_STEP_WORKLOADS:
+        sec = oracle_full_step_seconds(CONFIGS[name])
+        full[name] = {"wall_s": sec, "steps_per_s": 1.0 / sec}
+    return {"value": 1.0 / est if est > 0 else 0.0, "unit": "steps/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "method": "extrapolated: each operation timed on a slice of its rows and scaled "
+                      "to the whole step (a full step of this workload takes the oracle "
+                      f"~{est / 60:.0f} min)",
+            "sample": S.sample_desc(), "host_cores_available": cpu_cores(),
+            "full_step": dict(full, note="whole oracle steps measured end to end on the same "
+                                         "host, not extrapolated")}
+
+
 # ---------------------------------------------------------------------------- arms
 def run_reference(args, cfg, world, rank):
     if rank != 0:
@@ -280,54 +331,154 @@ def run_reference(args, cfg, world, rank):
     return 0
 
 
+def _source_digest(*paths) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in paths:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# kernel -> sources whose change makes a stored DRAM-traffic figure stale
+TRAFFIC_SOURCES = {
+    "tree_attention": ("medusa_head_speculative_02_b200/csrc/attention_tc.cu",
+                       "medusa_head_speculative_02_b200/csrc/common.cuh"),
+    "heads": ("medusa_head_speculative_02_b200/csrc/heads_tc.cu",
+              "medusa_head_speculative_02_b200/csrc/topk.cu",
+              "medusa_head_speculative_02_b200/csrc/common.cuh"),
+}
+
+
+def stored_traffic(workload: str, kernel: str, path: str | None = None):
+    """DRAM bytes (read + write) of one call of `kernel` at `workload`, from the
+    ncu capture summarised in profiles/dram_traffic.json; None when there is
+    none, or when the kernel's sources changed since it was taken."""
+    path = path or os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        e = json.load(open(path))[workload][kernel]
+    except Exception:
+        return None
+    if e.get("sources_sha16") != _source_digest(*TRAFFIC_SOURCES[kernel]):
+        return None
+    return e.get("bytes_per_call")
+
+
+def kernel_figures(cfg, st, calls, pk) -> dict:
+    """Back-to-back loops of the step's entry points on its own tensors."""
+    from medusa_head_speculative_02_b200 import kernel_bench as KB
+    out = {"heads": KB.time_heads(cfg, st.x, calls, ws=st.ws_heads, pk=pk),
+           "tree_attention": KB.time_attention(cfg, st.x, st.tree, calls, ws=st.ws_attn, pk=pk)}
+    if cfg.accept in ("greedy", "both"):
+        out["accept_greedy"] = KB.time_accept(cfg, st.vlogits, st.tree_tok, st.tree, calls,
+                                              typical=False, ws=st.ws_acc, pk=pk)
+    if cfg.accept in ("typical", "both"):
+        out["accept_typical"] = KB.time_accept(cfg, st.vlogits, st.tree_tok, st.tree, calls,
+                                               typical=True, ws=st.ws_acc, pk=pk)
+    # the bound that sets each kernel's floor: HBM bytes or tensor-core flops
+    for r in out.values():
+        if "algorithmic_flops" in r:
+            t_hbm = r["algorithmic_bytes"] / (pk["hbm_gbs"] * 1e9)
+            t_tc = r["algorithmic_flops"] / (pk["bf16_tflops"] * 1e12)
+            r["bound"] = "tensor" if t_tc > t_hbm else "hbm"
+            r["floor_ms"] = 1e3 * max(t_hbm, t_tc)
+        else:
+            r["bound"] = "hbm"
+            r["floor_ms"] = 1e3 * r["algorithmic_bytes"] / (pk["hbm_gbs"] * 1e9)
+    return out
+
+
+def roofline_of(name: str, r: dict, pk: dict, workload: str) -> dict:
+    """The JSON `roofline` object of kernel `name` from its kernel_figures entry."""
+    if r["bound"] == "tensor":
+        ach, peak, unit = r["tflops"], pk["bf16_tflops"], "TFLOP/s"
+    else:
+        ach, peak, unit = r["achieved"], pk["hbm_gbs"], "GB/s"
+    traffic = stored_traffic(workload, name)
+    line = {"kernel": name, "bound": r["bound"], "achieved": ach, "peak": peak, "unit": unit,
+            "frac": ach / peak, "traffic": traffic, "peak_src": pk["src"],
+            "avg_ms": r["avg_ms"], "calls": r["calls"],
+            "algorithmic_bytes": r["algorithmic_bytes"],
+            "timing": f"CUDA events around {r['calls']} back-to-back calls on the launching "
+                      f"stream, after the timed steps"}
+    if "algorithmic_flops" in r:
+        line.update({"algorithmic_flops": r["algorithmic_flops"], "tflops": r["tflops"],
+                     "tensor_frac": r["tensor_frac"],
+                     "tensor_frac_sustained": r["tensor_frac_sustained"],
+                     "hbm_frac": r["frac"]})
+    if traffic:
+        line["traffic_over_algorithmic"] = traffic / r["algorithmic_bytes"]
+    return line
+
+
+def time_steps(st, K, dev):
+    """Device time of K back-to-back verify steps (barrier + sync both sides)."""
+    stream = torch.cuda.current_stream(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for _ in range(K):
+        st.run()
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    return start.elapsed_time(end) / 1000.0
+
+
+def other_workloads(args, headline, dev, rank, pk) -> dict:
+    """Step rate and per-kernel figures of every other workload, one at a time
+    (each rank runs its own replica; figures are this rank's)."""
+    from medusa_head_speculative_02_b200.step import VerifyStep
+    names = CONFIG_ORDER if args.extra_configs == "all" else \
+        [n for n in args.extra_configs.split(",") if n and n != "none"]
+    res = {}
+    for name in names:
+        if name == headline:
+            continue
+        cfg = CONFIGS[name]
+        st = VerifyStep(cfg, dev, seed=rank)
+        for _ in range(5):
+            st.run()
+        torch.cuda.synchronize(dev)
+        t = time_steps(st, EXTRA_STEPS, dev)
+        kern = kernel_figures(cfg, st, KERNEL_CALLS, pk)
+        res[name] = {"steps_per_s": EXTRA_STEPS / t, "ms_per_step": 1e3 * t / EXTRA_STEPS,
+                     "steps": EXTRA_STEPS, "dtype": cfg.dtype, "batch": cfg.B,
+                     "kernels": {k: {kk: v[kk] for kk in ("avg_ms", "achieved", "unit", "frac",
+                                                         "bound", "floor_ms", "tflops",
+                                                         "tensor_frac", "key_chunks",
+                                                         "query_tiles_per_cta") if kk in v}
+                                 for k, v in kern.items()}}
+        del st
+        torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args, cfg, world, rank, local):
+    from medusa_head_speculative_02_b200 import kernel_bench as KB
     from medusa_head_speculative_02_b200.step import PipelinedHostIO, VerifyStep
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    pk = KB.peaks(ROOT)
     st = VerifyStep(cfg, dev, seed=rank)
-    stream = torch.cuda.current_stream(dev)
     for _ in range(args.warmup):
         st.run()
     torch.cuda.synchronize(dev)
 
+    # timed region: K steps back to back; clocks are sampled from just before
+    # it to the end of the per-kernel loops that follow
     K = args.steps
-    # The heads and attention calls of every EVENT_EVERY-th timed step are
-    # bracketed by CUDA events (the live roofline figures); the other steps
-    # run back to back, so the kernels of consecutive calls chain without an
-    # event between them.
-    sampled = list(range(0, K, EVENT_EVERY))
-    ev = {k: [torch.cuda.Event(enable_timing=True) for _ in range(4)] for k in sampled}
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
-    barrier()
-    torch.cuda.synchronize(dev)
-    start.record(stream)
-    for k in range(K):
-        e = ev.get(k)
-        if e is None:
-            st.run()
-            continue
-        e[0].record(stream)
-        st.heads()
-        e[1].record(stream)
-        st.build_tree()
-        e[2].record(stream)
-        st.attention()
-        e[3].record(stream)
-        st.accept()
-        st.compact()
-    end.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    clk = clocks.stop()
-    elapsed_s = start.elapsed_time(end) / 1000.0
-    heads_ms = statistics.mean(ev[k][0].elapsed_time(ev[k][1]) for k in sampled)
-    attn_ms = statistics.mean(ev[k][2].elapsed_time(ev[k][3]) for k in sampled)
+    elapsed_s = time_steps(st, K, dev)
     agg = aggregate(K, elapsed_s, world, dev)
     ms_per_step = agg["seconds"] * 1000.0 / K
     alen = st.accept_len.float().mean().item()
+    kern = kernel_figures(cfg, st, KERNEL_CALLS, pk)
+    clk = clocks.stop()
+    dominant = max(("heads", "tree_attention"), key=lambda k: kern[k]["avg_ms"])
 
     # end to end through the public API with host buffers: every step copies
     # its inputs from pinned host memory (the next step's on a copy stream,
@@ -340,6 +491,7 @@ def run_ours(args, cfg, world, rank, local):
         io.replay()
     torch.cuda.synchronize(dev)
     barrier()
+    stream = torch.cuda.current_stream(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(Ke // E2E_GRAPH_STEPS):
@@ -390,23 +542,14 @@ def run_ours(args, cfg, world, rank, local):
         pl = (None, cand[0, 1].view(cfg.B, cfg.K, cfg.s),
               cand[0, 0].view(torch.float32).view(cfg.B, cfg.K, cfg.s))
 
-        def one_rank():
+        def one_rank(_i=0):
             _api.medusa_heads_forward(st.x["h"], st.x["W1"], st.x["b1"], W2g, s=cfg.s,
                                       want_logits=False, out=pl, ws=ws)
             _api.medusa_topk_merge_planes(cand, cfg.s, offs, out=outs)
 
         one_rank()
         cand[1:] = cand[0]          # every shard's list slot holds a real list
-        for _ in range(3):
-            one_rank()
-        torch.cuda.synchronize(dev)
-        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        g0.record(stream)
-        for _ in range(SHARD_REPS):
-            one_rank()
-        g1.record(stream)
-        torch.cuda.synchronize(dev)
-        ms = g0.elapsed_time(g1) / SHARD_REPS
+        ms = KB.time_calls(one_rank, SHARD_REPS, device=dev)
         nbytes = st.heads_bytes() - elt * cfg.K * (cfg.V - (v1 - v0)) * cfg.d
         sharded[str(G)] = {"avg_ms": ms, "algorithmic_bytes": nbytes,
                            "achieved": nbytes / (ms / 1e3) / 1e9, "vocab_rows": v1 - v0}
@@ -439,27 +582,19 @@ def run_ours(args, cfg, world, rank, local):
         dec_alen = (grown.mean().item() / DECODE_STEPS) - 1.0
     dec = aggregate(DECODE_STEPS, dec_s if dec_err is None else 1.0, world, dev)
     del loop
+    torch.cuda.empty_cache()
 
-    peaks = measured_peaks()
-    attn_chunks = _api.attention_chunks(st.tree, cfg.B, cfg.Hq, cfg.Hkv, cfg.dh, cfg.Lcap,
-                                        cfg.torch_dtype)
-    attn_launches = _api.attention_launches(st.tree, cfg.B, cfg.Hq, cfg.Hkv, cfg.dh, cfg.Lcap,
-                                            cfg.torch_dtype)
-    attn_tiles = _api.attention_tiles_per_cta(st.tree, cfg.B, cfg.Hq, cfg.Hkv, cfg.dh, cfg.Lcap,
-                                              cfg.torch_dtype)
     sample_bytes = cfg.B * cfg.V * (4 if cfg.dtype == "f32" else 2)
     hb = st.heads_bytes()
     ab = st.attention_bytes()
-    af = st.attention_flops()
-    heads_gbs = hb / (heads_ms / 1000.0) / 1e9
-    attn_gbs = ab / (attn_ms / 1000.0) / 1e9
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "heads_traffic.json")
-    if os.path.exists(tpath):
-        try:
-            traffic = json.load(open(tpath)).get(cfg.name)
-        except Exception:
-            traffic = None
+    launches = st.launches_per_step()
+    io_h2d, io_d2h = io.h2d_bytes(), io.d2h_bytes()
+    # the oracle sampler takes host copies of this step's inputs
+    sampler = (OracleSampler(cfg, st.x, st.vlogits, target_ms=40.0)
+               if rank == 0 and world == 1 and not args.no_cpu_baseline else None)
+    del io, st
+    torch.cuda.empty_cache()
+    extra = other_workloads(args, cfg.name, dev, rank, pk)
 
     line = None
     if rank == 0:
@@ -473,41 +608,24 @@ def run_ours(args, cfg, world, rank, local):
                            "prefix": [cfg.L_lo, cfg.L_hi], "accept": cfg.accept,
                            "parallelism": f"dp{world} (independent replicas)",
                            "l2": "inputs larger than L2: each step streams "
-                                 f"{hb / 1e9:.2f} GB of head weights, evicting the "
-                                 f"{ab / 1e6:.1f} MB attention working set"},
+                                 f"{hb / 1e9:.2f} GB of head weights and "
+                                 f"{ab / 1e9:.2f} GB of K/V, evicting the 126 MB L2"},
                 "tokens_per_s": agg["value"] * cfg.B * (1.0 + alen),
                 "mean_accept_len": alen,
-                "roofline": {"kernel": "medusa_heads_forward (two heads_tc_kernel GEMMs + "
-                                       "top-s merge)",
-                             "timing": f"CUDA events around the heads call of every "
-                                       f"{EVENT_EVERY}th timed step ({len(sampled)} calls)",
-                             "bound": "hbm", "achieved": heads_gbs, "peak": peaks["hbm_gbs"],
-                             "unit": "GB/s", "frac": heads_gbs / peaks["hbm_gbs"],
-                             "traffic": traffic, "peak_src": peaks["src"],
-                             "algorithmic_bytes": hb, "avg_ms": heads_ms},
-                "kernels": {"tree_attention": {"achieved": attn_gbs, "unit": "GB/s",
-                                               "frac": attn_gbs / peaks["hbm_gbs"],
-                                               "algorithmic_bytes": ab, "avg_ms": attn_ms,
-                                               "tflops": af / (attn_ms / 1000.0) / 1e12,
-                                               "tensor_frac": af / (attn_ms / 1000.0) / 1e12
-                                               / peaks["bf16_tflops"],
-                                               "algorithmic_flops": af,
-                                               "key_chunks": attn_chunks,
-                                               "query_tiles_per_cta": attn_tiles,
-                                               "launches": attn_launches},
-                            "sample_next": {"avg_ms": sample_ms, "temperature": 0.7,
-                                            "algorithmic_bytes": sample_bytes,
-                                            "achieved": sample_bytes / (sample_ms / 1e3) / 1e9,
-                                            "unit": "GB/s",
-                                            "note": "one verify row per sequence; "
-                                                    "latency-bound at small batch"},
-                            "sharded_heads": {"per_shard_count": sharded, "unit": "GB/s",
-                                              "note": "one rank's heads for G vocabulary "
-                                                      "shards: replicated first projection, "
-                                                      "its W2 rows, merge of G candidate "
-                                                      "lists; the all-gather of G * B * K * s "
-                                                      "* 8 bytes between them is not "
-                                                      "included (needs G GPUs)"}},
+                "roofline": roofline_of(dominant, kern[dominant], pk, cfg.name),
+                "kernels": dict(kern, **{
+                    "sample_next": {"avg_ms": sample_ms, "temperature": 0.7,
+                                    "algorithmic_bytes": sample_bytes,
+                                    "achieved": sample_bytes / (sample_ms / 1e3) / 1e9,
+                                    "unit": "GB/s",
+                                    "note": "one verify row per sequence; latency-bound at "
+                                            "small batch"},
+                    "sharded_heads": {"per_shard_count": sharded, "unit": "GB/s",
+                                      "note": "one rank's heads for G vocabulary shards: "
+                                              "replicated first projection, its W2 rows, "
+                                              "merge of G candidate lists; the all-gather of "
+                                              "G * B * K * s * 8 bytes between them is not "
+                                              "included (needs G GPUs)"}}),
                 "decode_loop": ({"steps": DECODE_STEPS, "cuda_graph": True,
                                  "steps_per_s": dec["value"],
                                  "tokens_per_s": dec["value"] * cfg.B * (1.0 + dec_alen),
@@ -516,27 +634,20 @@ def run_ours(args, cfg, world, rank, local):
                                          "lengths; one captured step replayed per step"}
                                 if dec_err is None else {"error": dec_err}),
                 "e2e": {"value": e2e["value"], "unit": "steps/s",
-                        "h2d_bytes_per_step": io.h2d_bytes(),
-                        "d2h_bytes_per_step": io.d2h_bytes(), "steps": Ke,
+                        "h2d_bytes_per_step": io_h2d, "d2h_bytes_per_step": io_d2h,
+                        "steps": Ke,
                         "copies": "pinned host -> device every step; the next step's "
                                   "tree K/V slots, then its hidden state, queries, verify "
                                   "logits, roots and lengths, on a copy stream overlapping "
                                   "this step",
                         "launch": f"API calls and copies of {E2E_GRAPH_STEPS} steps captured "
                                   f"once into a CUDA graph, replayed"},
-                "gpu_launches": st.launches_per_step() * K,
-                "clocks": clk}
+                "gpu_launches": launches * K,
+                "clocks": dict(clk, window="timed steps and the per-kernel loops after them"),
+                "configs": extra}
     # CPU baseline: the oracle on rank 0 at N = 1 only
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        S = OracleSampler(cfg, st.x, st.vlogits, target_ms=40.0)
-        t0 = time.perf_counter()
-        while time.perf_counter() - t0 < args.cpu_seconds:
-            S.step()
-        est = S.estimate_step_seconds()
-        line["cpu_baseline"] = {"value": 1.0 / est if est > 0 else 0.0, "unit": "steps/s",
-                                "cores": blas_threads(), "kind": "oracle",
-                                "sample": S.sample_desc(),
-                                "host_cores_available": cpu_cores()}
+    if sampler is not None:
+        line["cpu_baseline"] = cpu_baseline(sampler, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
@@ -551,6 +662,9 @@ def main(argv=None):
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=list(CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--extra-configs", default="all",
+                    help="other workloads to report under `configs`: all, none, or a "
+                         "comma-separated list")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -12,7 +12,7 @@ import math
 
 import torch
 
-from . import api
+from . import api, kernel_bench
 from .synthetic import MedusaConfig, gen_inputs, plant_verify_logits
 
 # kernels this library launches per call
@@ -103,26 +103,18 @@ class VerifyStep:
         return (LAUNCHES["heads"] + LAUNCHES["build_tree"] + attn + n_acc * LAUNCHES["accept"] +
                 LAUNCHES["kv_compact"])
 
-    # algorithmic bytes --------------------------------------------------------
+    # algorithmic work ---------------------------------------------------------
     def heads_bytes(self) -> int:
-        c = self.cfg
-        e = 4 if c.dtype == "f32" else 2
-        return e * (c.K * c.d * c.d + c.K * c.d + c.K * c.V * c.d + c.B * c.d) + 8 * c.B * c.K * c.s
+        return kernel_bench.heads_bytes(self.cfg)
 
     def attention_flops(self) -> int:
         """Tensor-core work of the attention call: S = Q K^T and O = P V over
         every key of a sequence's prefix and tree slots, per query row."""
-        c = self.cfg
-        Lsum = int(self.x["prefix_len"].sum().item())
-        return 4 * c.Hq * c.N * (Lsum + c.B * c.N) * c.dh
+        return kernel_bench.attention_flops(self.cfg, int(self.x["prefix_len"].sum().item()))
 
     def attention_bytes(self) -> int:
         """K/V actually read (prefix + tree slots) + Q + O."""
-        c = self.cfg
-        e = 4 if c.dtype == "f32" else 2
-        Lsum = int(self.x["prefix_len"].sum().item())
-        kv = 2 * (Lsum + c.B * c.N) * c.Hkv * c.dh * e
-        return kv + 2 * c.B * c.N * c.Hq * c.dh * e
+        return kernel_bench.attention_bytes(self.cfg, int(self.x["prefix_len"].sum().item()))
 
 
 class HostIO:

@@ -97,8 +97,8 @@ def randn(shape, std: float, dtype, seed: int, tid: int, device,
     return out
 
 
-def gen_inputs(cfg: MedusaConfig, device="cpu", seed: int = 0) -> dict:
-    """All inputs of one verify step except the verify logits."""
+def gen_head_inputs(cfg: MedusaConfig, device="cpu", seed: int = 0) -> dict:
+    """Inputs of the heads and the tree expansion: h, W1, b1, W2, root_tok."""
     dt = cfg.torch_dtype
     x = {}
     x["h"] = randn((cfg.B, cfg.d), 1.0, dt, seed, _TID["h"], device)
@@ -108,12 +108,27 @@ def gen_inputs(cfg: MedusaConfig, device="cpu", seed: int = 0) -> dict:
     g = generator(seed, _TID["root"], device)
     x["root_tok"] = torch.randint(0, cfg.V, (cfg.B,), generator=g, device=device,
                                   dtype=torch.int64).to(torch.int32)
+    return x
+
+
+def gen_attention_inputs(cfg: MedusaConfig, device="cpu", seed: int = 0) -> dict:
+    """Inputs of the tree attention and the compaction: prefix_len, q, k_cache,
+    v_cache (the same values gen_inputs gives for the same seed)."""
+    dt = cfg.torch_dtype
+    x = {}
     g = generator(seed, _TID["L"], device)
     x["prefix_len"] = torch.randint(cfg.L_lo, cfg.L_hi + 1, (cfg.B,), generator=g,
                                     device=device, dtype=torch.int64).to(torch.int32)
     x["q"] = randn((cfg.B, cfg.N, cfg.Hq, cfg.dh), 1.0, dt, seed, _TID["q"], device)
     x["k_cache"] = randn((cfg.B, cfg.Lcap, cfg.Hkv, cfg.dh), 1.0, dt, seed, _TID["k"], device)
     x["v_cache"] = randn((cfg.B, cfg.Lcap, cfg.Hkv, cfg.dh), 1.0, dt, seed, _TID["v"], device)
+    return x
+
+
+def gen_inputs(cfg: MedusaConfig, device="cpu", seed: int = 0) -> dict:
+    """All inputs of one verify step except the verify logits."""
+    x = gen_head_inputs(cfg, device, seed)
+    x.update(gen_attention_inputs(cfg, device, seed))
     return x
 
 

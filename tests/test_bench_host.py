@@ -1,0 +1,55 @@
+"""CPU: host-side logic of bench.py's measurement lines (roofline object,
+stored DRAM traffic and its staleness check, per-kernel work formulas)."""
+import json
+
+import pytest
+
+import bench
+from medusa_head_speculative_02_b200 import kernel_bench as KB
+from medusa_head_speculative_02_b200.synthetic import CONFIGS
+
+PK = {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0,
+      "src": "measured"}
+
+
+def test_roofline_hbm_and_tensor_bound():
+    r = {"avg_ms": 1.0, "calls": 50, "algorithmic_bytes": 3.25e9, "achieved": 3250.0,
+         "frac": 0.5, "bound": "hbm", "algorithmic_flops": 8e11, "tflops": 800.0,
+         "tensor_frac": 0.5, "tensor_frac_sustained": 800 / 1400}
+    line = bench.roofline_of("tree_attention", r, PK, "no_such_workload")
+    assert line["unit"] == "GB/s" and line["peak"] == 6500.0
+    assert line["frac"] == pytest.approx(0.5) and line["traffic"] is None
+    r["bound"] = "tensor"
+    line = bench.roofline_of("tree_attention", r, PK, "no_such_workload")
+    assert line["unit"] == "TFLOP/s" and line["frac"] == pytest.approx(0.5)
+    assert line["hbm_frac"] == pytest.approx(0.5)
+
+
+def test_stored_traffic_goes_stale_when_sources_change(tmp_path):
+    digest = bench._source_digest(*bench.TRAFFIC_SOURCES["tree_attention"])
+    path = tmp_path / "t.json"
+    path.write_text(json.dumps({"w": {"tree_attention": {"bytes_per_call": 123,
+                                                         "sources_sha16": digest}}}))
+    assert bench.stored_traffic("w", "tree_attention", str(path)) == 123
+    path.write_text(json.dumps({"w": {"tree_attention": {"bytes_per_call": 123,
+                                                         "sources_sha16": "0" * 16}}}))
+    assert bench.stored_traffic("w", "tree_attention", str(path)) is None
+    assert bench.stored_traffic("other", "tree_attention", str(path)) is None
+
+
+def test_work_formulas_at_the_long_context_workload():
+    c = CONFIGS["longctx_b4"]
+    Lsum = c.B * c.L_hi
+    # K and V of prefix + tree slots, Q read and O written
+    kv = 2 * (Lsum + c.B * c.N) * c.Hkv * c.dh * 2
+    assert KB.attention_bytes(c, Lsum) == kv + 2 * c.B * c.N * c.Hq * c.dh * 2
+    assert KB.attention_flops(c, Lsum) == 4 * c.Hq * c.N * (Lsum + c.B * c.N) * c.dh
+    assert KB.heads_bytes(c) == 2 * (c.K * c.d * c.d + c.K * c.d + c.K * c.V * c.d + c.B * c.d) \
+        + 8 * c.B * c.K * c.s
+    assert KB.accept_bytes(c) == c.B * c.N * c.V * 2
+
+
+def test_rotation_copies():
+    assert KB._copies(10 * KB.L2_BYTES) == 1
+    assert KB._copies(KB.L2_BYTES // 4) == 12
+    assert KB._copies(1) == 16
