@@ -39,7 +39,8 @@ sampled next token is drawn from the last accepted node's row by Gumbel-max
 with SplitMix64 noise keyed by (seed, call offset, sequence, vocab index);
 candidate lists of vocabulary shards merge in the top-s order of the whole
 row (value desc, global id asc), so a merge of per-shard top-s lists equals
-the top-s of the unsplit row.
+the top-s of the unsplit row; the layers of a multi-layer verification
+share the tree, the prefix lengths and the accepted path.
 
 Parity: every function here is pinned by tests/test_oracle_pins.py against
 closed forms, library routines or brute force (see each docstring).
@@ -57,6 +58,7 @@ __all__ = [
     "typical_row_stats", "typical_threshold", "accept_typical", "kv_compact",
     "ancestors_or_self", "heads_hidden", "heads_logits", "splitmix64",
     "uniform01", "gumbel32", "sample_next", "temperature_by_depth", "topk_merge",
+    "tree_attention_layers", "kv_compact_layers",
 ]
 
 
@@ -415,6 +417,35 @@ def kv_compact(k_cache, v_cache, prefix_len, accept_len, accept_nodes):
             v_new[b, L[b] + j] = v_old[b, L[b] + nodes[b, j]]
         new_len[b] = L[b] + 1 + A[b]
     return k_new, v_new, new_len
+
+
+# ---------------------------------------------------------------------------
+# Several layers.  [MD] "ツリーアテンションによる並列検証": the whole candidate
+# tree is verified in one forward pass of the base model, i.e. every layer
+# runs the masked attention over its own cache with the same tree and prefix
+# lengths, and after acceptance every layer's cache keeps the accepted path.
+# READING: the layers share the tree, the prefix lengths and the accepted
+# path; each has its own queries and K/V cache.
+# ---------------------------------------------------------------------------
+def tree_attention_layers(q, k_caches, v_caches, prefix_len, plan, scale, rows=None):
+    """q [layers][B][N][Hq][dh]; k_caches, v_caches [layers][B][Lcap][Hkv][dh].
+    Layer l's output is tree_attention over layer l's queries and cache;
+    returns [layers][...] (the shape tree_attention gives for ``rows``)."""
+    return np.stack([tree_attention(q[l], k_caches[l], v_caches[l], prefix_len, plan, scale,
+                                    rows=rows) for l in range(q.shape[0])])
+
+
+def kv_compact_layers(k_caches, v_caches, prefix_len, accept_len, accept_nodes):
+    """The accepted path compacted in every layer's cache ([layers][B][Lcap]
+    [Hkv][dh]); returns (new_k, new_v, new_len), new_len being the same for
+    every layer."""
+    ks, vs, new_len = [], [], None
+    for l in range(k_caches.shape[0]):
+        k, v, new_len = kv_compact(k_caches[l], v_caches[l], prefix_len, accept_len,
+                                   accept_nodes)
+        ks.append(k)
+        vs.append(v)
+    return np.stack(ks), np.stack(vs), new_len
 
 
 # ---------------------------------------------------------------------------

@@ -549,3 +549,67 @@ def test_topk_merge_pads_when_candidates_run_out():
     idxs = np.array([[[4, -1]], [[9, -1]]])
     mi, mv = O.topk_merge(vals, idxs, 3)
     assert mi.tolist() == [[4, 9, -1]] and mv[0, 0] == 3.0 and np.isnan(mv[0, 2])
+
+
+# ----------------------------------------------------------------------------
+# Several layers
+# ----------------------------------------------------------------------------
+def test_attention_layers_chain_tree_is_causal_attention_per_layer():
+    """Three layers, a chain tree (s = 1): each layer's rows equal ordinary
+    causal attention (torch SDPA) over that layer's own prefix + chain."""
+    nl, B, K, L, Hq, Hkv, dh = 3, 2, 5, 40, 4, 2, 16
+    N = K + 1
+    g = torch.Generator().manual_seed(21)
+    q = torch.randn(nl, B, N, Hq, dh, generator=g, dtype=torch.float64)
+    kc = torch.randn(nl, B, L + N, Hkv, dh, generator=g, dtype=torch.float64)
+    vc = torch.randn(nl, B, L + N, Hkv, dh, generator=g, dtype=torch.float64)
+    plan = O.tree_plan(K, 1, N)
+    got = O.tree_attention_layers(q, kc, vc, [L] * B, plan, 0.25)
+    G = Hq // Hkv
+    for l in range(nl):
+        qf = torch.zeros(B, Hq, L + N, dh, dtype=torch.float64)
+        qf[:, :, L:] = q[l].permute(0, 2, 1, 3)
+        kf = kc[l].repeat_interleave(G, dim=2).permute(0, 2, 1, 3)
+        vf = vc[l].repeat_interleave(G, dim=2).permute(0, 2, 1, 3)
+        ref = F.scaled_dot_product_attention(qf, kf, vf, is_causal=True, scale=0.25)
+        assert np.allclose(got[l], ref[:, :, L:].permute(0, 2, 1, 3).numpy(), atol=1e-12)
+
+
+def test_attention_layers_follow_their_own_caches():
+    """Swapping two layers' queries and caches swaps their outputs, and a
+    layer's output depends on no other layer (doubling layer 0's V doubles
+    its output and leaves layer 1's)."""
+    nl, B, L, Hq, dh = 2, 1, 30, 2, 8
+    plan = O.tree_plan(3, 2, 9)
+    g = torch.Generator().manual_seed(4)
+    q = torch.randn(nl, B, 9, Hq, dh, generator=g, dtype=torch.float64)
+    kc = torch.randn(nl, B, L + 9, Hq, dh, generator=g, dtype=torch.float64)
+    vc = torch.randn(nl, B, L + 9, Hq, dh, generator=g, dtype=torch.float64)
+    a = O.tree_attention_layers(q, kc, vc, [L], plan, 0.3)
+    b = O.tree_attention_layers(q.flip(0), kc.flip(0), vc.flip(0), [L], plan, 0.3)
+    assert np.array_equal(a, b[::-1])
+    vc2 = vc.clone()
+    vc2[0] *= 2.0          # attention is linear in V: layer 0 doubles, layer 1 stays
+    c = O.tree_attention_layers(q, kc, vc2, [L], plan, 0.3)
+    assert np.array_equal(a[1], c[1]) and np.allclose(c[0], 2.0 * a[0], atol=1e-12)
+
+
+def test_kv_compact_layers_equals_gather_in_every_layer():
+    """Every layer's slots L_b + j take old slots L_b + nodes[j] (numpy
+    fancy-index gather), new_len = L_b + 1 + a, other slots untouched."""
+    nl, B, Lcap, Hkv, dh, K = 3, 2, 30, 2, 4, 3
+    rng = np.random.default_rng(8)
+    kc = rng.standard_normal((nl, B, Lcap, Hkv, dh))
+    vc = rng.standard_normal((nl, B, Lcap, Hkv, dh))
+    L = np.array([10, 4])
+    A = np.array([3, 1])
+    nodes = np.array([[0, 2, 5, 9], [0, 1, -1, -1]])
+    nk, nv, nlen = O.kv_compact_layers(kc, vc, L, A, nodes)
+    assert (nlen == L + 1 + A).all()
+    for b in range(B):
+        dst = L[b] + np.arange(1, A[b] + 1)
+        src = L[b] + nodes[b, 1:A[b] + 1]
+        ek, ev = kc.copy(), vc.copy()
+        ek[:, b, dst] = kc[:, b, src]
+        ev[:, b, dst] = vc[:, b, src]
+        assert np.array_equal(nk[:, b], ek[:, b]) and np.array_equal(nv[:, b], ev[:, b])
