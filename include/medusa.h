@@ -297,8 +297,10 @@ int medusa_accept_typical_per_head(const void* vlogits, int dtype,
  * which every GPU that loads the library holds until the process exits.
  * Limit: B * N <= MEDUSA_NOALLOC_ACCEPT_PARTS, else MEDUSA_ERR_INVALID_ARG
  * and nothing is launched.  The first call on a device looks up the array's
- * device address (cudaGetSymbolAddress, host side, once per device); make
- * that first call before any stream capture.  All calls share the array:
+ * device address (cudaGetSymbolAddress, host side, once per device and
+ * context: after a cudaDeviceReset the next call looks it up again in the
+ * new context); make that first call before any stream capture.  All calls
+ * share the array:
  * calls that may overlap on the GPU (different streams without ordering)
  * race and must be serialized by the caller.  No memory is allocated or
  * freed by this call.

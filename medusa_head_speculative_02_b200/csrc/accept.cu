@@ -399,20 +399,52 @@ static __device__ __align__(256) RowPart g_accept_scratch[MEDUSA_NOALLOC_ACCEPT_
 namespace {
 std::mutex g_scratch_mu;
 RowPart* g_scratch_addr[64] = {nullptr};
+unsigned long long g_scratch_ctx[64] = {0};  // id of the context the address belongs to
 
-// Device address of g_accept_scratch on the current device, looked up once
-// per device (with that device current) and cached.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Id of the CUDA context current on this thread (the driver never reuses an
+// id within a process, unlike a context handle); false when no context is
+// current yet or the driver entry points are unavailable.
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = (CtxGetCurrentFn)p;
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = (CtxGetIdFn)p;
+  });
+  CUcontext ctx = nullptr;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_accept_scratch on the current device.  Looked up with
+// that device current on its first call, and again whenever the device's
+// context has changed since (a cudaDeviceReset destroys the context the
+// cached address belonged to); otherwise the cached address is used.
 int scratch_address(RowPart** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= 64) return fail(MEDUSA_ERR_UNSUPPORTED, "device ordinal >= 64");
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  unsigned long long id = 0;
+  const bool have_id = current_context_id(&id);
+  if (!g_scratch_addr[dev] || !have_id || id != g_scratch_ctx[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_accept_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_accept_scratch)");
     g_scratch_addr[dev] = (RowPart*)p;
+    g_scratch_ctx[dev] = current_context_id(&id) ? id : 0ull;
   }
   *out = g_scratch_addr[dev];
   return MEDUSA_OK;
@@ -429,15 +461,12 @@ int accept_greedy_noalloc_launch(const void* vlog, int dtype, const int32_t* tok
     return fail(MEDUSA_ERR_INVALID_ARG,
                 "medusa_accept_greedy_noalloc: B*N exceeds its static scratch "
                 "(MEDUSA_NOALLOC_ACCEPT_PARTS rows)");
-  AccPlan P = make_plan((int)rows, V);
-  if (rows * P.splits > MEDUSA_NOALLOC_ACCEPT_PARTS) {
-    // fewer, longer chunks per row so every (row, chunk) result fits
-    const int splits = (int)(MEDUSA_NOALLOC_ACCEPT_PARTS / rows);
-    int chunk = (V + splits - 1) / splits;
-    chunk = (chunk + 7) & ~7;
-    P.chunk = chunk;
-    P.splits = (V + chunk - 1) / chunk;
-  }
+  const AccPlan P = make_plan((int)rows, V);
+  // make_plan splits rows only while rows < 4 x SMs, so rows x splits stays
+  // below 4 x SMs + rows, far inside the array for any device
+  if (rows * P.splits > MEDUSA_NOALLOC_ACCEPT_PARTS)
+    return fail(MEDUSA_ERR_UNSUPPORTED,
+                "medusa_accept_greedy_noalloc: row chunks exceed the static scratch");
   RowPart* parts = nullptr;
   int rc = scratch_address(&parts);
   if (rc) return rc;
