@@ -455,6 +455,40 @@ def other_workloads(args, headline, dev, rank, pk) -> dict:
     return res
 
 
+MULTI_LAYER = ("7b_b1", 32)   # workload and layer count of the multi-layer verification figure
+
+
+def multi_layer_figure(dev, rank, pk) -> dict:
+    """A verify step through 32 attention layers at the 7B shape: heads,
+    tree, one tree-attention call per layer (each on its own queries and
+    cache), acceptance, one compaction over every layer's cache."""
+    from medusa_head_speculative_02_b200 import kernel_bench as KB
+    from medusa_head_speculative_02_b200.step import MultiLayerStep
+    name, layers = MULTI_LAYER
+    cfg = CONFIGS[name]
+    ml = MultiLayerStep(cfg, layers, dev, seed=rank)
+    for _ in range(3):
+        ml.run()
+    torch.cuda.synchronize(dev)
+    steps = 20
+    barrier()
+    t = time_steps(ml, steps, dev)
+    prefix_sum = int(ml.st.x["prefix_len"].sum().item())
+    ab = KB.attention_bytes(cfg, prefix_sum) * layers
+    att_ms = KB.time_calls(lambda i: ml.attention(), 10, device=dev)
+    res = {"workload": name, "layers": layers, "steps": steps,
+           "steps_per_s": steps / t, "ms_per_step": 1e3 * t / steps,
+           "attention_ms_all_layers": att_ms,
+           "attention_achieved_gbs": ab / (att_ms / 1e3) / 1e9,
+           "attention_frac": ab / (att_ms / 1e3) / 1e9 / pk["hbm_gbs"],
+           "launches_per_step": ml.launches_per_step(),
+           "note": "one medusa_tree_attention call per layer on its own cache, then one "
+                   "medusa_kv_compact_layers over all layers"}
+    del ml
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args, cfg, world, rank, local):
     from medusa_head_speculative_02_b200 import kernel_bench as KB
     from medusa_head_speculative_02_b200.step import PipelinedHostIO, VerifyStep
@@ -595,6 +629,12 @@ def run_ours(args, cfg, world, rank, local):
     del io, st
     torch.cuda.empty_cache()
     extra = other_workloads(args, cfg.name, dev, rank, pk)
+    multi = None
+    if not args.no_multi_layer:
+        try:
+            multi = multi_layer_figure(dev, rank, pk)
+        except Exception as ex:  # reported in the line, the main result stands
+            multi = {"error": f"{type(ex).__name__}: {ex}"[:300]}
 
     line = None
     if rank == 0:
@@ -644,7 +684,8 @@ def run_ours(args, cfg, world, rank, local):
                                   f"once into a CUDA graph, replayed"},
                 "gpu_launches": launches * K,
                 "clocks": dict(clk, window="timed steps and the per-kernel loops after them"),
-                "configs": extra}
+                "configs": extra,
+                "multi_layer": multi}
     # CPU baseline: the oracle on rank 0 at N = 1 only
     if sampler is not None:
         line["cpu_baseline"] = cpu_baseline(sampler, args.cpu_seconds)
@@ -662,6 +703,8 @@ def main(argv=None):
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=list(CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--no-multi-layer", action="store_true",
+                    help="skip the multi-layer verification figure")
     ap.add_argument("--extra-configs", default="all",
                     help="other workloads to report under `configs`: all, none, or a "
                          "comma-separated list")

@@ -52,7 +52,8 @@ typedef enum {
   MEDUSA_ERR_INVALID_ARG = -1, /* null pointer, bad size, bad tree, ... */
   MEDUSA_ERR_UNSUPPORTED = -2, /* valid but not implemented (dtype/shape) */
   MEDUSA_ERR_CUDA = -3,        /* a CUDA runtime/driver call failed */
-  MEDUSA_ERR_TIMEOUT = -4      /* a device-side bounded wait ran out */
+  MEDUSA_ERR_TIMEOUT = -4,     /* a device-side bounded wait ran out */
+  MEDUSA_ERR_BOUNDS = -5       /* a device-side index check failed (debug build) */
 } medusa_status;
 
 typedef enum { MEDUSA_F32 = 0, MEDUSA_BF16 = 1 } medusa_dtype;
@@ -73,8 +74,20 @@ const char* medusa_version(void);
 
 /*
  * Reads (and with clear != 0 resets) the device status word of the current
- * device.  Synchronizes the device.  *status receives MEDUSA_OK or
- * MEDUSA_ERR_TIMEOUT.  Returns MEDUSA_ERR_CUDA if the device is unusable.
+ * device.  Synchronizes the device.  *status receives MEDUSA_OK,
+ * MEDUSA_ERR_TIMEOUT or, from the debug build, MEDUSA_ERR_BOUNDS (then
+ * medusa_last_error() names the first failing check site).  Returns
+ * MEDUSA_ERR_CUDA if the device is unusable.
+ *
+ * Debug build (libmedusa_debug.so, compiled with MEDUSA_DEBUG; the Python
+ * binding loads it when the environment has MEDUSA_DEBUG=1): every kernel
+ * also checks the indices it derives from its inputs (tree slots against the
+ * cache, nodes against N, tokens against V, plan entries against K s).  A
+ * failed check records MEDUSA_ERR_BOUNDS in the status word and skips the
+ * access (it never traps).  Sites: 1 tree expansion (head, rank) index,
+ * 2 attention key tile, 3 attention key slot (SIMT kernel), 4 acceptance
+ * parent, 5 acceptance tree token, 6 compaction node, 7 sampling node,
+ * 8 shard-merge candidate id.  Results of the release build are identical.
  */
 int medusa_device_status(int* status, int clear);
 
@@ -325,6 +338,24 @@ int medusa_kv_compact(void* k_cache, void* v_cache, const int32_t* prefix_len,
                       const int32_t* accept_len, const int32_t* accept_nodes,
                       int B, int Hkv, int dh, int Lcap, int K, int dtype,
                       int32_t* new_len, void* stream);
+
+/*
+ * medusa_kv_compact over the caches of n_layers layers in one launch.
+ * [MD] "ツリーアテンションによる並列検証": the tree is verified in one forward
+ * pass of the base model, so every layer has written the tree's K/V at slots
+ * L_b..L_b+N-1 of its own cache, and the accepted path is kept in each.
+ * Layer l's caches start at k_caches + l * layer_stride and v_caches + l *
+ * layer_stride (elements of dtype; layer_stride >= B * Lcap * Hkv * dh when
+ * n_layers > 1), each [B][Lcap][Hkv][dh].  prefix_len, accept_len,
+ * accept_nodes and new_len are shared by the layers (new_len written once).
+ * Same rules and skipped entries as medusa_kv_compact; n_layers = 1 is
+ * medusa_kv_compact.
+ */
+int medusa_kv_compact_layers(void* k_caches, void* v_caches, int n_layers,
+                             long long layer_stride, const int32_t* prefix_len,
+                             const int32_t* accept_len, const int32_t* accept_nodes,
+                             int B, int Hkv, int dh, int Lcap, int K, int dtype,
+                             int32_t* new_len, void* stream);
 
 /* ------------------------------------------------------------------------
  * Merge of top-s candidate lists from G vocabulary shards (heads whose W2

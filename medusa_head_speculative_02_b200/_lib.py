@@ -1,6 +1,9 @@
 """ctypes loader for libmedusa.so (the C ABI of include/medusa.h).
 
-Loading fails loudly: there is no CPU or Python fallback for any call.
+With MEDUSA_DEBUG=1 in the environment the MEDUSA_DEBUG build
+(libmedusa_debug.so: device-side index checks reported as
+MEDUSA_ERR_BOUNDS) is loaded instead.  Loading fails loudly: there is no CPU
+or Python fallback for any call.
 """
 from __future__ import annotations
 
@@ -8,9 +11,10 @@ import ctypes as C
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmedusa.so")
+DEBUG = os.environ.get("MEDUSA_DEBUG", "0") == "1"
+LIB_PATH = os.path.join(_HERE, "libmedusa_debug.so" if DEBUG else "libmedusa.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, -1, -2, -3, -4
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = 0, -1, -2, -3, -4, -5
 F32, BF16 = 0, 1
 MAX_K, MAX_S, MAX_N = 8, 16, 256
 
@@ -48,6 +52,8 @@ SIGNATURES = {
                                             csz, vp]),
     "medusa_accept_greedy_noalloc": (ci, [vp, ci, vp, vp, ci, ci, vp, vp, vp, vp]),
     "medusa_kv_compact": (ci, [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, vp, vp]),
+    "medusa_kv_compact_layers": (ci, [vp, vp, ci, C.c_longlong, vp, vp, vp, ci, ci, ci, ci, ci,
+                                      ci, vp, vp]),
 }
 
 _lib = None

@@ -334,6 +334,28 @@ def medusa_sample_next(vlogits, accept_len, accept_nodes, temperature: float, se
     return out
 
 
+def medusa_kv_compact_layers(k_caches, v_caches, prefix_len, accept_len, accept_nodes, K: int,
+                             new_len=None):
+    """Compaction of the accepted path in every layer's cache: k_caches,
+    v_caches [layers][B][Lcap][Hkv][dh] (contiguous, so the layer stride is
+    one layer's cache); returns new_len [B]."""
+    nl, B, Lcap, Hkv, dh = k_caches.shape
+    _need(k_caches, "k_caches")
+    _need(v_caches, "v_caches", k_caches.dtype, k_caches.shape)
+    _need(prefix_len, "prefix_len", torch.int32, (B,))
+    _need(accept_len, "accept_len", torch.int32, (B,))
+    _need(accept_nodes, "accept_nodes", torch.int32, (B, K + 1))
+    new_len = torch.empty(B, dtype=torch.int32, device=k_caches.device) if new_len is None \
+        else new_len
+    L.check(L.lib().medusa_kv_compact_layers(_ptr(k_caches), _ptr(v_caches), nl,
+                                             B * Lcap * Hkv * dh, _ptr(prefix_len),
+                                             _ptr(accept_len), _ptr(accept_nodes), B, Hkv, dh,
+                                             Lcap, K, _dt(k_caches), _ptr(new_len),
+                                             _stream(k_caches.device)),
+            "medusa_kv_compact_layers")
+    return new_len
+
+
 def medusa_kv_compact(k_cache, v_cache, prefix_len, accept_len, accept_nodes, K: int,
                       new_len=None):
     B, Lcap, Hkv, dh = k_cache.shape

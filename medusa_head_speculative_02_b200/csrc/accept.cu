@@ -269,7 +269,10 @@ __global__ void __launch_bounds__(MEDUSA_MAX_N)
   if (n > 0 && n < N) {
     const int par = parent[n];
     const int t = tok[(size_t)b * N + n];
-    if (TYPICAL) {
+    dbg_ok(t >= 0 && t < V, DBG_ACCEPT_TOKEN);  // a token outside the vocabulary never matches
+    if (!dbg_ok(par >= 0 && par < n, DBG_ACCEPT_PARENT)) {
+      c = false;
+    } else if (TYPICAL) {
       if (t >= 0 && t < V) {
         const float x = to_f32(vlog[((size_t)b * N + par) * V + t]);
         // the parent's row was reduced at the scale of n's depth

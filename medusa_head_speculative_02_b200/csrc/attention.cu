@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(kThreads)
       const int j = e / DH, dd = e - j * DH;
       const int key = t0 + j;
       float kv = 0.f, vv = 0.f;
-      if (key < k_hi) {
+      if (key < k_hi && dbg_ok(slot0 + key < Lcap, DBG_ATTN_SLOT)) {
         const size_t off = (((size_t)b * Lcap + slot0 + key) * Hkv + kvh) * DH + dd;
         kv = to_f32(kc[off]);
         vv = to_f32(vc[off]);

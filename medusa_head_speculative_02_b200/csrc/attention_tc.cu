@@ -407,6 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < T; ++j) {
         const int st = j % kStages;
         const int key0 = j < rg.n_pre ? rg.k_lo + j * BN : Lb + (j - rg.n_pre) * BN;
+        dbg_ok(key0 >= 0 && key0 < Lb + p.N && key0 < p.Lcap, DBG_ATTN_KEY_TILE);
         const int z = b * p.Lcap + key0;
         if (!mbar_wait(&emp[st], ((uint32_t)(j / kStages) & 1u) ^ 1u, abort_flag)) break;
         mbar_arrive_expect_tx(&ful[st], TILE);
@@ -823,6 +824,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < T; ++j) {
         const int st = j % stages;
         const int key0 = j < rg.n_pre ? rg.k_lo + j * BN : Lb + (j - rg.n_pre) * BN;
+        dbg_ok(key0 >= 0 && key0 < Lb + p.N && key0 < p.Lcap, DBG_ATTN_KEY_TILE);
         const int z = b * p.Lcap + key0;
         if (!mbar_wait(&emp[st], ((uint32_t)(j / stages) & 1u) ^ 1u, abort_flag)) break;
         mbar_arrive_expect_tx(&ful[st], TILE);

@@ -10,9 +10,40 @@
 namespace medusa {
 
 // ---------------------------------------------------------------- status word
-// Set by a bounded device wait that ran out; read by medusa_device_status().
-enum : unsigned { DEV_OK = 0u, DEV_TIMEOUT = 1u };
+// Set by a bounded device wait that ran out (DEV_TIMEOUT) or, in MEDUSA_DEBUG
+// builds, by a failed index check (DEV_BOUNDS); read by medusa_device_status().
+enum : unsigned { DEV_OK = 0u, DEV_TIMEOUT = 1u, DEV_BOUNDS = 2u };
 extern __device__ unsigned int g_dev_status;
+// First failing check site of a MEDUSA_DEBUG build (0: none).
+extern __device__ unsigned int g_dev_debug_site;
+
+// Check sites of the MEDUSA_DEBUG build (reported by medusa_debug_site()).
+enum : unsigned {
+  DBG_TREE_HEAD_RANK = 1u,   // tree expansion: plan's (head, rank) index outside [0, K s)
+  DBG_ATTN_KEY_TILE = 2u,    // attention: a staged key tile starts outside the sequence
+  DBG_ATTN_SLOT = 3u,        // SIMT attention: a key slot outside the cache
+  DBG_ACCEPT_PARENT = 4u,    // acceptance: parent node outside [0, N)
+  DBG_ACCEPT_TOKEN = 5u,     // acceptance: a tree token outside [0, V)
+  DBG_COMPACT_NODE = 6u,     // compaction: accepted node outside the tree / cache
+  DBG_SAMPLE_NODE = 7u,      // sampling: last accepted node outside [0, N)
+  DBG_MERGE_SHARD = 8u       // shard merge: a candidate id below -1
+};
+
+// Device-side index check.  MEDUSA_DEBUG builds: when `ok` is false the
+// status word gets DEV_BOUNDS, the first failing site is kept, and the
+// caller skips the access (the check never traps).  Other builds: always
+// true, no code.
+#ifdef MEDUSA_DEBUG
+__device__ __forceinline__ bool dbg_ok(bool ok, unsigned site) {
+  if (!ok) {
+    atomicOr(&g_dev_status, DEV_BOUNDS);
+    atomicCAS(&g_dev_debug_site, 0u, site);
+  }
+  return ok;
+}
+#else
+__device__ __forceinline__ constexpr bool dbg_ok(bool, unsigned) { return true; }
+#endif
 
 // Wall-clock bound of every device-side spin wait (ns).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;

@@ -175,9 +175,11 @@ int accept_greedy_noalloc_launch(const void* vlog, int dtype, const int32_t* tok
                                  int32_t* accept_nodes, int32_t* next_tok, cudaStream_t st);
 
 // ---------------------------------------------------------------- compaction
+// layers caches, layer_stride elements apart (1 layer: stride unused)
 int kv_compact_launch(void* k, void* v, const int32_t* L, const int32_t* alen,
                       const int32_t* anodes, int B, int Hkv, int dh, int Lcap, int K,
-                      int dtype, int32_t* new_len, cudaStream_t st);
+                      int dtype, int32_t* new_len, cudaStream_t st, int layers = 1,
+                      long long layer_stride = 0);
 
 // ---------------------------------------------------------------- TMA descriptors
 // Encodes a bf16 tensor map (dims innermost first) with 128-byte swizzling.

@@ -2,6 +2,7 @@
 // validation, the tree plan, TMA descriptor encoding and the device status.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cstring>
@@ -17,6 +18,7 @@
 namespace medusa {
 
 __device__ unsigned int g_dev_status = 0u;
+__device__ unsigned int g_dev_debug_site = 0u;
 
 namespace {
 thread_local std::string t_last_error;
@@ -53,6 +55,15 @@ int fail(int code, const std::string& msg) {
 int cuda_fail(cudaError_t e, const char* what) {
   return fail(MEDUSA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
 }
+
+// NVTX range around one ABI call (shows the call by name in Nsight Systems
+// and Nsight Compute range filters); a no-op unless a tool is attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 int num_sms() {
   static std::atomic<int> cache[64];
@@ -240,21 +251,32 @@ int medusa_selftest_wait_timeout(int limit_ms, void* stream) {
 
 const char* medusa_last_error(void) { return t_last_error.c_str(); }
 
-const char* medusa_version(void) { return "medusa-b200 0.1 (sm_100a)"; }
+#ifdef MEDUSA_DEBUG
+const char* medusa_version(void) { return "medusa-b200 0.2 (sm_100a, MEDUSA_DEBUG index checks)"; }
+#else
+const char* medusa_version(void) { return "medusa-b200 0.2 (sm_100a)"; }
+#endif
 
 int medusa_device_status(int* status, int clear) {
   if (!status) return fail(MEDUSA_ERR_INVALID_ARG, "status is NULL");
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
-  unsigned int v = 0;
+  unsigned int v = 0, site = 0;
   e = cudaMemcpyFromSymbol(&v, g_dev_status, sizeof(v));
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&site, g_dev_debug_site, sizeof(site));
   if (e != cudaSuccess) return cuda_fail(e, "read device status");
   if (clear) {
     const unsigned int z = 0;
     e = cudaMemcpyToSymbol(g_dev_status, &z, sizeof(z));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_dev_debug_site, &z, sizeof(z));
     if (e != cudaSuccess) return cuda_fail(e, "clear device status");
   }
-  *status = (v & DEV_TIMEOUT) ? MEDUSA_ERR_TIMEOUT : MEDUSA_OK;
+  if (v & DEV_BOUNDS) {
+    *status = MEDUSA_ERR_BOUNDS;
+    fail(MEDUSA_ERR_BOUNDS, "device index check failed, first at site " + std::to_string(site));
+  } else {
+    *status = (v & DEV_TIMEOUT) ? MEDUSA_ERR_TIMEOUT : MEDUSA_OK;
+  }
   return MEDUSA_OK;
 }
 
@@ -275,6 +297,7 @@ int medusa_tree_plan_host(int K, int s, int N, int32_t* parent, int32_t* depth,
 }
 
 int medusa_tree_create(int K, int s, int N, medusa_tree_t** out) {
+  medusa::NvtxRange nvtx_range("medusa_tree_create");
   if (!out) return fail(MEDUSA_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
   medusa_tree* t = nullptr;
@@ -358,6 +381,7 @@ int medusa_heads_forward(const void* h, const void* W1, const void* b1, const vo
                          int d, int V, int K, int dtype, float* logits, int s,
                          int32_t* topk_idx, float* topk_val, void* ws, size_t ws_bytes,
                          void* stream) {
+  medusa::NvtxRange nvtx_range("medusa_heads_forward");
   if (!dtype_ok(dtype)) return fail(MEDUSA_ERR_INVALID_ARG, "bad dtype");
   if (B < 0 || d <= 0 || V <= 0 || K < 1 || K > MEDUSA_MAX_K)
     return fail(MEDUSA_ERR_INVALID_ARG, "bad heads shape");
@@ -382,6 +406,7 @@ int medusa_heads_forward(const void* h, const void* W1, const void* b1, const vo
 
 int medusa_topk(const void* logits, int dtype, int R, int V, int s, int32_t* idx, float* val,
                 void* stream) {
+  medusa::NvtxRange nvtx_range("medusa_topk");
   if (!dtype_ok(dtype)) return fail(MEDUSA_ERR_INVALID_ARG, "bad dtype");
   if (R < 0 || V < 1) return fail(MEDUSA_ERR_INVALID_ARG, "bad shape");
   if (s < 1 || s > MEDUSA_MAX_S || s > V)
@@ -393,6 +418,7 @@ int medusa_topk(const void* logits, int dtype, int R, int V, int s, int32_t* idx
 int medusa_build_tree(const medusa_tree_t* tree, const int32_t* root_tok,
                       const int32_t* topk_idx, const int32_t* prefix_len, int B,
                       int32_t* tree_tok, int32_t* tree_pos, void* stream) {
+  medusa::NvtxRange nvtx_range("medusa_build_tree");
   int rc = check_tree(tree);
   if (rc) return rc;
   if (B < 0) return fail(MEDUSA_ERR_INVALID_ARG, "B < 0");
@@ -433,6 +459,7 @@ int medusa_tree_attention(const void* q, const void* k_cache, const void* v_cach
                           const int32_t* prefix_len, const medusa_tree_t* tree, int B, int Hq,
                           int Hkv, int dh, int Lcap, float scale, int dtype, void* out, void* ws,
                           size_t ws_bytes, void* stream) {
+  medusa::NvtxRange nvtx_range("medusa_tree_attention");
   int rc = check_tree(tree);
   if (rc) return rc;
   if (!dtype_ok(dtype)) return fail(MEDUSA_ERR_INVALID_ARG, "bad dtype");
@@ -505,6 +532,7 @@ int medusa_accept_greedy(const void* vlogits, int dtype, const int32_t* tree_tok
                          const medusa_tree_t* tree, int B, int V, int32_t* accept_len,
                          int32_t* accept_nodes, int32_t* next_tok, void* ws, size_t ws_bytes,
                          void* stream) {
+  medusa::NvtxRange nvtx_range("medusa_accept_greedy");
   return accept_common(vlogits, dtype, tree_tok, tree, B, V, false, 1.f, nullptr, 0.f, 0.f,
                        accept_len, accept_nodes, next_tok, ws, ws_bytes, stream);
 }
@@ -513,6 +541,7 @@ int medusa_accept_typical(const void* vlogits, int dtype, const int32_t* tree_to
                           const medusa_tree_t* tree, int B, int V, float temperature, float eps,
                           float delta, int32_t* accept_len, int32_t* accept_nodes,
                           int32_t* next_tok, void* ws, size_t ws_bytes, void* stream) {
+  medusa::NvtxRange nvtx_range("medusa_accept_typical");
   return accept_common(vlogits, dtype, tree_tok, tree, B, V, true, temperature, nullptr, eps,
                        delta, accept_len, accept_nodes, next_tok, ws, ws_bytes, stream);
 }
@@ -522,6 +551,7 @@ int medusa_accept_typical_per_head(const void* vlogits, int dtype, const int32_t
                                    const float* temperatures, float eps, float delta,
                                    int32_t* accept_len, int32_t* accept_nodes, int32_t* next_tok,
                                    void* ws, size_t ws_bytes, void* stream) {
+  medusa::NvtxRange nvtx_range("medusa_accept_typical_per_head");
   if (!temperatures) return fail(MEDUSA_ERR_INVALID_ARG, "temperatures is NULL");
   return accept_common(vlogits, dtype, tree_tok, tree, B, V, true, 1.f, temperatures, eps,
                        delta, accept_len, accept_nodes, next_tok, ws, ws_bytes, stream);
@@ -530,6 +560,7 @@ int medusa_accept_typical_per_head(const void* vlogits, int dtype, const int32_t
 int medusa_accept_greedy_noalloc(const void* vlogits, int dtype, const int32_t* tree_tok,
                                  const medusa_tree_t* tree, int B, int V, int32_t* accept_len,
                                  int32_t* accept_nodes, int32_t* next_tok, void* stream) {
+  medusa::NvtxRange nvtx_range("medusa_accept_greedy_noalloc");
   int rc = check_tree(tree);
   if (rc) return rc;
   if (!dtype_ok(dtype)) return fail(MEDUSA_ERR_INVALID_ARG, "bad dtype");
@@ -544,6 +575,7 @@ int medusa_accept_greedy_noalloc(const void* vlogits, int dtype, const int32_t* 
 int medusa_kv_compact(void* k_cache, void* v_cache, const int32_t* prefix_len,
                       const int32_t* accept_len, const int32_t* accept_nodes, int B, int Hkv,
                       int dh, int Lcap, int K, int dtype, int32_t* new_len, void* stream) {
+  medusa::NvtxRange nvtx_range("medusa_kv_compact");
   if (!dtype_ok(dtype)) return fail(MEDUSA_ERR_INVALID_ARG, "bad dtype");
   if (B < 0 || Hkv <= 0 || dh <= 0 || Lcap <= 0 || K < 0 || K > MEDUSA_MAX_K)
     return fail(MEDUSA_ERR_INVALID_ARG, "bad shape");
@@ -556,9 +588,31 @@ int medusa_kv_compact(void* k_cache, void* v_cache, const int32_t* prefix_len,
                            Lcap, K, dtype, new_len, (cudaStream_t)stream);
 }
 
+int medusa_kv_compact_layers(void* k_caches, void* v_caches, int n_layers,
+                             long long layer_stride, const int32_t* prefix_len,
+                             const int32_t* accept_len, const int32_t* accept_nodes, int B,
+                             int Hkv, int dh, int Lcap, int K, int dtype, int32_t* new_len,
+                             void* stream) {
+  medusa::NvtxRange nvtx_range("medusa_kv_compact_layers");
+  if (!dtype_ok(dtype)) return fail(MEDUSA_ERR_INVALID_ARG, "bad dtype");
+  if (n_layers < 0 || B < 0 || Hkv <= 0 || dh <= 0 || Lcap <= 0 || K < 0 || K > MEDUSA_MAX_K)
+    return fail(MEDUSA_ERR_INVALID_ARG, "bad shape");
+  if (((size_t)Hkv * dh * (dtype == MEDUSA_F32 ? 4 : 2)) % 4 != 0)
+    return fail(MEDUSA_ERR_UNSUPPORTED, "slot size must be a multiple of 4 bytes");
+  if (n_layers > 1 && layer_stride < (long long)B * Lcap * Hkv * dh)
+    return fail(MEDUSA_ERR_INVALID_ARG, "layer_stride smaller than one layer's cache");
+  if (B == 0 || n_layers == 0) return MEDUSA_OK;
+  if (!k_caches || !v_caches || !prefix_len || !accept_len || !accept_nodes)
+    return fail(MEDUSA_ERR_INVALID_ARG, "NULL pointer");
+  return kv_compact_launch(k_caches, v_caches, prefix_len, accept_len, accept_nodes, B, Hkv, dh,
+                           Lcap, K, dtype, new_len, (cudaStream_t)stream, n_layers,
+                           n_layers > 1 ? layer_stride : 0);
+}
+
 int medusa_topk_merge(const float* val, const int32_t* idx, long long shard_stride,
                       const int32_t* v0, int G, int R, int c, int s, int32_t* out_idx,
                       float* out_val, void* stream) {
+  medusa::NvtxRange nvtx_range("medusa_topk_merge");
   if (G < 1 || R < 0 || c < 1 || s < 1 || s > MEDUSA_MAX_S || (long long)G * c > (1LL << 30))
     return fail(MEDUSA_ERR_INVALID_ARG, "bad shape");
   if (shard_stride < (long long)R * c) return fail(MEDUSA_ERR_INVALID_ARG, "shard_stride < R * c");
@@ -572,6 +626,7 @@ int medusa_sample_next(const void* vlogits, int dtype, const int32_t* accept_len
                        const int32_t* accept_nodes, int B, int N, int V, int K,
                        float temperature, uint64_t seed, uint64_t offset,
                        const uint64_t* offset_dev, int32_t* next_tok, void* stream) {
+  medusa::NvtxRange nvtx_range("medusa_sample_next");
   if (!dtype_ok(dtype)) return fail(MEDUSA_ERR_INVALID_ARG, "bad dtype");
   if (B < 0 || N <= 0 || N > MEDUSA_MAX_N || V <= 0 || K < 0 || K > MEDUSA_MAX_K)
     return fail(MEDUSA_ERR_INVALID_ARG, "bad shape");

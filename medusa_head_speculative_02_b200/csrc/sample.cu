@@ -57,6 +57,7 @@ __global__ void __launch_bounds__(kThreads)
   const int a = alen[b];
   const int node = (a >= 0 && a <= K) ? anodes[(size_t)b * (K + 1) + a] : -1;
   const bool valid = node >= 0 && node < N;  // uniform over the cluster
+  if (part == 0 && threadIdx.x == 0) dbg_ok(valid, DBG_SAMPLE_NODE);
   uint64_t best = 0ull;
   if (valid) {
     const T* row = vlog + ((size_t)b * N + node) * (size_t)V;

@@ -122,7 +122,10 @@ __global__ void __launch_bounds__(kThreads)
     const int g = t / c, j = t - g * c;
     const size_t o = (size_t)g * (size_t)gs + (size_t)row * c + j;
     const int i = idx[o];
-    if (i < 0) continue;
+    if (i < 0) {
+      dbg_ok(i == -1, DBG_MERGE_SHARD);  // -1 marks an empty slot; lower ids are malformed
+      continue;
+    }
     const uint64_t key = make_key(val[o], (uint32_t)(i + (v0 ? v0[g] : 0)));
     if (key > kth) topk_insert<kSmax>(k, s, key, kth);
   }

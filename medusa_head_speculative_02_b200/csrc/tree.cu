@@ -22,6 +22,7 @@ __global__ void build_tree_kernel(const int32_t* __restrict__ head_rank,
   if (i >= B * N) return;
   const int b = i / N, n = i - b * N;
   const int hr = head_rank[n];
+  if (!dbg_ok(hr >= -1 && hr < Ks, DBG_TREE_HEAD_RANK)) return;
   tok[i] = hr < 0 ? root[b] : topk[(size_t)b * Ks + hr];
   if (pos) pos[i] = L[b] + depth[n];
 }

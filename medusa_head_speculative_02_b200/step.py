@@ -117,6 +117,57 @@ class VerifyStep:
         return kernel_bench.attention_bytes(self.cfg, int(self.x["prefix_len"].sum().item()))
 
 
+class MultiLayerStep:
+    """A verify step through `layers` attention layers: heads (+ top-s), tree
+    expansion, one tree-attention call per layer on that layer's queries and
+    cache (the tree, prefix lengths and workspace shared), acceptance, and
+    one compaction of the accepted path over every layer's cache.  The
+    per-layer queries and caches are synthetic (no base model): layer l
+    draws them from its own seed."""
+
+    def __init__(self, cfg: MedusaConfig, layers: int, device="cuda", seed: int = 0):
+        from .synthetic import gen_attention_inputs
+        self.st = VerifyStep(cfg, device, seed)
+        self.layers = layers
+        c = cfg
+        dev = self.st.dev
+        self.q = torch.empty(layers, c.B, c.N, c.Hq, c.dh, dtype=c.torch_dtype, device=dev)
+        self.k = torch.empty(layers, c.B, c.Lcap, c.Hkv, c.dh, dtype=c.torch_dtype, device=dev)
+        self.v = torch.empty_like(self.k)
+        for l in range(layers):
+            xl = gen_attention_inputs(c, dev, seed * 1000 + l)
+            self.q[l].copy_(xl["q"])
+            self.k[l].copy_(xl["k_cache"])
+            self.v[l].copy_(xl["v_cache"])
+            del xl
+        self.out = torch.empty_like(self.q)
+
+    def attention(self):
+        st = self.st
+        for l in range(self.layers):
+            api.medusa_tree_attention(self.q[l], self.k[l], self.v[l], st.x["prefix_len"],
+                                      st.tree, st.scale, out=self.out[l], ws=st.ws_attn)
+
+    def compact(self):
+        st = self.st
+        api.medusa_kv_compact_layers(self.k, self.v, st.x["prefix_len"], st.accept_len,
+                                     st.accept_nodes, st.cfg.K, new_len=st.new_len)
+
+    def run(self):
+        self.st.heads()
+        self.st.build_tree()
+        self.attention()
+        self.st.accept()
+        self.compact()
+
+    def launches_per_step(self) -> int:
+        c = self.st.cfg
+        attn = api.attention_launches(self.st.tree, c.B, c.Hq, c.Hkv, c.dh, c.Lcap, c.torch_dtype)
+        n_acc = 2 if c.accept == "both" else 1
+        return (LAUNCHES["heads"] + LAUNCHES["build_tree"] + self.layers * attn +
+                n_acc * LAUNCHES["accept"] + LAUNCHES["kv_compact"])
+
+
 class HostIO:
     """Pinned host copies of one step's per-step inputs and outputs."""
 

@@ -35,6 +35,16 @@ def test_version_string():
     assert b"sm_100a" in L.lib().medusa_version()
 
 
+def test_debug_library_exports_every_declared_symbol():
+    """libmedusa_debug.so (MEDUSA_DEBUG index checks) has the same ABI."""
+    path = os.path.join(os.path.dirname(L.LIB_PATH), "libmedusa_debug.so")
+    dbg = C.CDLL(path)
+    for n in _declared_symbols():
+        assert hasattr(dbg, n), n
+    dbg.medusa_version.restype = C.c_char_p
+    assert b"MEDUSA_DEBUG" in dbg.medusa_version()
+
+
 @pytest.mark.parametrize("name", list(CONFIGS))
 def test_host_tree_plan_matches_oracle(name):
     cfg = CONFIGS[name]
