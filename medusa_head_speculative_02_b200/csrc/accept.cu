@@ -87,12 +87,22 @@ template <> struct Lanes<float> {
 };
 
 // Running per-thread state of the row reduction: the argmax (value, first
-// index) and, for typical acceptance, (m, Z, S) of z = x * zscale in base 2.
+// index) and, for typical acceptance, (m, Z, S) of z = x * zscale in base 2,
+// Z and S kept as two packed fp32 lanes (even / odd columns of each load)
+// so the sums run as two independent chains of f32x2 operations; folded
+// into sf at the end.
 struct RedState {
   float bv;
   int bi;
   Soft sf;
+  unsigned long long Z2, S2;
 };
+
+__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 
 // Folds NV consecutive logits starting at column `base` (indices increase
 // from call to call within a thread, so a strict > keeps the first maximum).
@@ -112,22 +122,36 @@ __device__ __forceinline__ void red_consume(RedState& st, const float (&x)[NV], 
   if (TYPICAL) {
     const float vz = vm * zscale;  // zscale > 0: the max of the scaled values
     if (vz > st.sf.m) {
-      if (st.sf.Z > 0.f) {
-        const float d = st.sf.m - vz;  // < 0
+      if (st.sf.m != -INFINITY) {
+        // S <- c (d Z + S), Z <- c Z on both lanes, c = 2^d (d < 0)
+        const float d = st.sf.m - vz;
         const float c = ex2_approx(d);
-        st.sf.S = c * fmaf(d, st.sf.Z, st.sf.S);
-        st.sf.Z *= c;
+        const unsigned long long d2 = f2_pack(d, d), c2 = f2_pack(c, c);
+        st.S2 = f2_mul(c2, f2_fma(d2, st.Z2, st.S2));
+        st.Z2 = f2_mul(c2, st.Z2);
       }
       st.sf.m = vz;
     }
     if (st.sf.m != -INFINITY) {  // else every value so far is -inf: nothing to add
-#pragma unroll
-      for (int j = 0; j < NV; ++j) {
-        // t <= 0; clamped so that a -inf (or NaN) logit adds 0 to Z and S
-        const float t = fmaxf(fmaf(x[j], zscale, -st.sf.m), -200.f);
+      const unsigned long long zs2 = f2_pack(zscale, zscale);
+      const unsigned long long nm2 = f2_pack(-st.sf.m, -st.sf.m);
+      if (NV == 1) {  // unaligned rows: one logit at a time, on lane 0
+        const float t = fmaxf(fmaf(x[0], zscale, -st.sf.m), -200.f);
         const float e = ex2_approx(t);
-        st.sf.Z += e;
-        st.sf.S = fmaf(e, t, st.sf.S);
+        st.Z2 = f2_add(st.Z2, f2_pack(e, 0.f));
+        st.S2 = f2_fma(f2_pack(e, 0.f), f2_pack(t, 0.f), st.S2);
+        return;
+      }
+#pragma unroll
+      for (int j = 0; j + 1 < NV; j += 2) {
+        // t <= 0; clamped so that a -inf (or NaN) logit adds 0 to Z and S
+        float t0, t1;
+        f2_unpack(f2_fma(f2_pack(x[j], x[(j + 1) % NV]), zs2, nm2), t0, t1);
+        t0 = fmaxf(t0, -200.f);
+        t1 = fmaxf(t1, -200.f);
+        const unsigned long long e2 = f2_pack(ex2_approx(t0), ex2_approx(t1));
+        st.Z2 = f2_add(st.Z2, e2);
+        st.S2 = f2_fma(e2, f2_pack(t0, t1), st.S2);
       }
     }
   }
@@ -152,7 +176,7 @@ __global__ void __launch_bounds__(kRedThreads)
   const int hi = min(V, lo + chunk);
   const T* xr = vlog + row * (size_t)V;
   constexpr int VEC = Lanes<T>::n;
-  RedState st{-INFINITY, 0x7FFFFFFF, Soft{-INFINITY, 0.f, 0.f}};
+  RedState st{-INFINITY, 0x7FFFFFFF, Soft{-INFINITY, 0.f, 0.f}, 0ull, 0ull};
   const bool vec_ok = ((((uintptr_t)(xr + lo)) & 15u) == 0) && ((hi - lo) % VEC == 0);
   if (vec_ok) {
     const uint4* p = reinterpret_cast<const uint4*>(xr + lo);
@@ -188,6 +212,13 @@ __global__ void __launch_bounds__(kRedThreads)
   }
   uint64_t best = make_key(st.bv, (uint32_t)st.bi);
   Soft sf = st.sf;
+  if (TYPICAL) {  // both lanes share sf.m
+    float z0, z1, s0, s1;
+    f2_unpack(st.Z2, z0, z1);
+    f2_unpack(st.S2, s0, s1);
+    sf.Z = z0 + z1;
+    sf.S = s0 + s1;
+  }
   // block reduction
   best = warp_max_u64(best);
   if (TYPICAL) {
