@@ -157,13 +157,19 @@ size_t medusa_heads_workspace_size(int B, int d, int V, int K, int s, int dtype)
  *            by logit descending, ties to the lower id;
  *   topk_val [B][K][s] fp32 (only written when topk_idx is non-NULL).
  * bf16: W1 and W2 are streamed by tcgen05 tensor-core GEMMs (TMA-fed, fp32
- * accumulation in TMEM) with the bias, SiLU and residual fused in the first
- * GEMM's epilogue and a partial top-s fused in the second's.  The hidden
- * activation u is passed to the second GEMM as a bf16 hi/lo pair (u = hi +
- * lo), so it keeps ~16 mantissa bits.  fp32: SIMT kernels.
- * Limits: d % 8 == 0; B <= 32 (bf16) or 16 (fp32); K <= MEDUSA_MAX_K;
- * 1 <= s <= MEDUSA_MAX_S, s <= V.  Pointers 16-byte aligned.
+ * accumulation in TMEM) with the bias, SiLU and residual applied between
+ * the two GEMMs and a partial top-s fused in the second's epilogue.  The
+ * hidden activation u is passed to the second GEMM as a bf16 hi/lo pair (u =
+ * hi + lo), so it keeps ~16 mantissa bits.  B <= 32: weight-streaming
+ * kernels (activations as a narrow N operand, HBM-bound).  32 < B <=
+ * MEDUSA_MAX_HEADS_B: compute-bound kernels with N = 256 activation columns
+ * per tile (the second GEMM executes 2x the method's flops, for hi and lo).
+ * fp32: SIMT kernels.
+ * Limits: d % 8 == 0; B <= MEDUSA_MAX_HEADS_B (bf16) or 16 (fp32);
+ * K <= MEDUSA_MAX_K; 1 <= s <= MEDUSA_MAX_S, s <= V.  Pointers 16-byte
+ * aligned.
  */
+#define MEDUSA_MAX_HEADS_B 4096
 int medusa_heads_forward(const void* h, const void* W1, const void* b1,
                          const void* W2, int B, int d, int V, int K, int dtype,
                          float* logits, int s, int32_t* topk_idx,

@@ -231,11 +231,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int tile, sp, kh, mt, k0, k1;
       unit_coords(p, unit, tile, sp, kh, mt, k0, k1);
       const uint32_t acc = local & 1u;
-      mbar_wait(&tfull[acc], (local >> 1) & 1u, abort_flag);
-      // The four epilogue warps leave together if any wait ran out, so none
-      // can be left behind at a named barrier.
-      named_bar_sync(1, 128);
-      if (*abort_flag) break;
+      const bool good = mbar_wait(&tfull[acc], (local >> 1) & 1u, abort_flag);
+      // The four epilogue warps leave together if any wait ran out (one
+      // decision, the OR of every thread's view), so none can be left
+      // behind at a named barrier.
+      if (bar_red_or(1, 128, !good || *abort_flag)) break;
       tc_fence_after();
       float v[NC];
 #pragma unroll

@@ -101,6 +101,9 @@ struct HeadsArgs {
 };
 size_t heads_tc_workspace(int B, int d, int V, int K, int s);
 int heads_tc_launch(const HeadsArgs& a, cudaStream_t st);
+// large batch (bf16, B > 32): compute-bound GEMMs with N = 256 (csrc/heads_big.cu)
+size_t heads_big_workspace(int B, int d, int V, int K, int s);
+int heads_big_launch(const HeadsArgs& a, cudaStream_t st);
 size_t heads_simt_workspace(int B, int d, int V, int K, int s);
 int heads_simt_launch(const HeadsArgs& a, cudaStream_t st);
 

@@ -373,8 +373,8 @@ int medusa_tree_info(const medusa_tree_t* t, int* K, int* s, int* N, int32_t* pa
 size_t medusa_heads_workspace_size(int B, int d, int V, int K, int s, int dtype) {
   if (B <= 0 || d <= 0 || V <= 0 || K <= 0 || s < 0) return 0;
   if (s == 0) s = 1;
-  return dtype == MEDUSA_BF16 ? heads_tc_workspace(B, d, V, K, s)
-                              : heads_simt_workspace(B, d, V, K, s);
+  if (dtype != MEDUSA_BF16) return heads_simt_workspace(B, d, V, K, s);
+  return B > 32 ? heads_big_workspace(B, d, V, K, s) : heads_tc_workspace(B, d, V, K, s);
 }
 
 int medusa_heads_forward(const void* h, const void* W1, const void* b1, const void* W2, int B,
@@ -394,14 +394,16 @@ int medusa_heads_forward(const void* h, const void* W1, const void* b1, const vo
   if (!aligned16(h) || !aligned16(W1) || !aligned16(W2) || (b1 && !aligned16(b1)) ||
       !aligned16(ws))
     return fail(MEDUSA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
-  if (dtype == MEDUSA_BF16 && B > 32) return fail(MEDUSA_ERR_UNSUPPORTED, "bf16 heads: B <= 32");
+  if (dtype == MEDUSA_BF16 && B > MEDUSA_MAX_HEADS_B)
+    return fail(MEDUSA_ERR_UNSUPPORTED, "bf16 heads: B <= MEDUSA_MAX_HEADS_B");
   if (dtype == MEDUSA_F32 && B > 16) return fail(MEDUSA_ERR_UNSUPPORTED, "fp32 heads: B <= 16");
   if (B == 0) return MEDUSA_OK;
   const size_t need = medusa_heads_workspace_size(B, d, V, K, s, dtype);
   if (!ws || ws_bytes < need) return fail(MEDUSA_ERR_INVALID_ARG, "workspace too small");
   HeadsArgs a{h, W1, b1, W2, B, d, V, K, dtype, logits, s, topk_idx, topk_val, ws, ws_bytes};
   cudaStream_t st = (cudaStream_t)stream;
-  return dtype == MEDUSA_BF16 ? heads_tc_launch(a, st) : heads_simt_launch(a, st);
+  if (dtype != MEDUSA_BF16) return heads_simt_launch(a, st);
+  return B > 32 ? heads_big_launch(a, st) : heads_tc_launch(a, st);
 }
 
 int medusa_topk(const void* logits, int dtype, int R, int V, int s, int32_t* idx, float* val,
