@@ -456,6 +456,30 @@ def other_workloads(args, headline, dev, rank, pk) -> dict:
 
 
 MULTI_LAYER = ("7b_b1", 32)   # workload and layer count of the multi-layer verification figure
+LARGE_BATCH = ("7b_b1", 256)  # workload shape and batch of the compute-bound heads figure
+
+
+def heads_large_batch_figure(dev, pk) -> dict:
+    """The heads at B = 256 sequences with the 7B shapes (d = 4096, V =
+    32000, K = 5): tensor-bound GEMMs.  `tflops` counts the method's
+    multiply-adds x 2; `executed_tflops` also the second GEMM's doubled
+    columns (u as the bf16 hi/lo pair), which is what the tensor pipe runs."""
+    from medusa_head_speculative_02_b200 import kernel_bench as KB
+    from medusa_head_speculative_02_b200.synthetic import gen_head_inputs
+    name, B = LARGE_BATCH
+    c = CONFIGS[name].scaled(B=B)
+    x = gen_head_inputs(c, dev, 0)
+    r = KB.time_heads(c, x, 20, pk=pk)
+    exe = 2 * c.B * c.K * c.d * c.d + 2 * (2 * c.B) * c.K * c.V * c.d
+    r.update({"workload": f"{name} heads at B = {B}", "batch": B,
+              "executed_flops": exe,
+              "executed_tflops": exe / (r["avg_ms"] / 1e3) / 1e12,
+              "executed_tensor_frac_sustained": exe / (r["avg_ms"] / 1e3) / 1e12
+              / pk["bf16_tflops_sustained"],
+              "kernel": "heads_big2_kernel (cta_group::2, M = 256, N = 256) x 2 + SiLU + top-s merge"})
+    del x
+    torch.cuda.empty_cache()
+    return r
 
 
 def multi_layer_figure(dev, rank, pk) -> dict:
@@ -487,6 +511,62 @@ def multi_layer_figure(dev, rank, pk) -> dict:
     del ml
     torch.cuda.empty_cache()
     return res
+
+
+def run_tensor_parallel(args, cfg, world, rank, local):
+    """--heads vocab-shard: one batch of B sequences served by all ranks.
+    The heads' second projection is split by vocabulary rows (one NCCL
+    all-gather of every rank's [values; ids] candidate planes, B * K * s * 8
+    bytes per rank, then the merge kernel), the tree attention and the
+    compaction by kv-head (Hkv / N heads of every sequence per rank, no
+    exchange), the acceptance replicated.  Whole-job throughput = verify
+    steps/s of the one batch (strong scaling: the work per step is fixed)."""
+    from medusa_head_speculative_02_b200 import kernel_bench as KB
+    from medusa_head_speculative_02_b200.sharded import ShardedHeads, shard_w2, vocab_shard
+    from medusa_head_speculative_02_b200.step import VerifyStep
+    if cfg.Hkv % world or cfg.Hq % world:
+        raise SystemExit(f"--heads vocab-shard: {world} ranks must divide the kv-heads ({cfg.Hkv})")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    pk = KB.peaks(ROOT)
+    lcfg = cfg.scaled(Hq=cfg.Hq // world, Hkv=cfg.Hkv // world)
+    st = VerifyStep(lcfg, dev, seed=0)   # identical heads inputs and verify logits on every rank
+    v0, v1 = vocab_shard(cfg.V, world, rank)
+    st.x["W2"] = shard_w2(st.x["W2"], world, rank)
+    torch.cuda.empty_cache()
+    sh = ShardedHeads(st.x["W1"], st.x["b1"], st.x["W2"], cfg.V, cfg.B, cfg.s)
+    st.heads = lambda: sh(st.x["h"], out=(st.topk_idx, st.topk_val))
+    for _ in range(args.warmup):
+        st.run()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    elapsed_s = time_steps(st, K, dev)
+    t = max_over_ranks(elapsed_s, dev)
+    attn = KB.time_attention(lcfg, st.x, st.tree, KERNEL_CALLS, ws=st.ws_attn, pk=pk)
+    heads = KB.time_heads(lcfg.scaled(V=v1 - v0), st.x, KERNEL_CALLS, pk=pk)
+    clk = clocks.stop()
+    if rank == 0:
+        line = {"metric": METRIC, "value": K / t, "unit": "steps/s", "n_gpus": world, "steps": K,
+                "warmup": args.warmup, "ms_per_step": 1e3 * t / K, "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": cfg.name, "batch": cfg.B, "d": cfg.d, "vocab": cfg.V,
+                           "heads": cfg.K, "top_s": cfg.s, "tree_nodes": cfg.N,
+                           "q_heads": cfg.Hq, "kv_heads": cfg.Hkv, "head_dim": cfg.dh,
+                           "prefix": [cfg.L_lo, cfg.L_hi], "accept": cfg.accept,
+                           "parallelism": f"tp{world}: W2 split by vocabulary (one all-gather of "
+                                          f"{cfg.B * cfg.K * cfg.s * 8} B per rank per step), "
+                                          f"attention and compaction by kv-head "
+                                          f"({cfg.Hkv // world} per rank), acceptance replicated"},
+                "tokens_per_s": K / t * cfg.B * (1.0 + st.accept_len.float().mean().item()),
+                "roofline": roofline_of("tree_attention", attn, pk, cfg.name + f"/tp{world}"),
+                "kernels": {"heads_rank_share": heads, "tree_attention_rank_share": attn},
+                "gpu_launches": (st.launches_per_step() + 1) * K,
+                "clocks": dict(clk, window="timed steps and the per-kernel loops after them")}
+        print(json.dumps(line), flush=True)
+    return 0
 
 
 def run_ours(args, cfg, world, rank, local):
@@ -629,6 +709,10 @@ def run_ours(args, cfg, world, rank, local):
     del io, st
     torch.cuda.empty_cache()
     extra = other_workloads(args, cfg.name, dev, rank, pk)
+    try:
+        big = heads_large_batch_figure(dev, pk)
+    except Exception as ex:  # reported in the line, the main result stands
+        big = {"error": f"{type(ex).__name__}: {ex}"[:300]}
     multi = None
     if not args.no_multi_layer:
         try:
@@ -660,6 +744,7 @@ def run_ours(args, cfg, world, rank, local):
                                     "unit": "GB/s",
                                     "note": "one verify row per sequence; latency-bound at "
                                             "small batch"},
+                    "heads_large_batch": big,
                     "sharded_heads": {"per_shard_count": sharded, "unit": "GB/s",
                                       "note": "one rank's heads for G vocabulary shards: "
                                               "replicated first projection, its W2 rows, "
@@ -703,6 +788,10 @@ def main(argv=None):
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=list(CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--heads", choices=["replicas", "vocab-shard"], default="replicas",
+                    help="replicas: every rank serves its own sequences (weak scaling); "
+                         "vocab-shard: all ranks serve one batch, heads split by vocabulary "
+                         "and attention by kv-head (strong scaling)")
     ap.add_argument("--no-multi-layer", action="store_true",
                     help="skip the multi-layer verification figure")
     ap.add_argument("--extra-configs", default="all",
@@ -720,6 +809,10 @@ def main(argv=None):
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
     try:
+        if args.heads == "vocab-shard":
+            if world < 2:
+                raise SystemExit("--heads vocab-shard needs torchrun with 2 or more ranks")
+            return run_tensor_parallel(args, cfg, world, rank, local)
         return run_ours(args, cfg, world, rank, local)
     finally:
         if world > 1:

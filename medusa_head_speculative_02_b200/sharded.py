@@ -72,9 +72,15 @@ def gather_candidates(local: torch.Tensor, group=None, out: torch.Tensor | None 
 class ShardedHeads:
     """Per-rank state of the vocabulary-sharded heads for fixed (B, K, s, V):
     the W2 slice, the candidate and gather buffers, the shard offsets on the
-    device and the heads workspace, all allocated once."""
+    device and the heads workspace, all allocated once.
 
-    def __init__(self, W1, b1, W2_shard, V: int, B: int, s: int, group=None, align: int = 128):
+    `local_fn(h, W1, b1, W2_shard, s, idx, val)` fills this rank's top-s of
+    its slice and `merge_fn(gathered, s, v0, out_idx, out_val)` merges the
+    gathered planes; both default to the library calls
+    (medusa_heads_forward, medusa_topk_merge_planes)."""
+
+    def __init__(self, W1, b1, W2_shard, V: int, B: int, s: int, group=None, align: int = 128,
+                 local_fn=None, merge_fn=None):
         self.group = group
         self.G = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
@@ -87,15 +93,26 @@ class ShardedHeads:
             raise ValueError(f"s={s} exceeds the {Vr} rows of rank {self.rank}'s shard")
         self.W1, self.b1, self.W2 = W1, b1, W2_shard
         self.K = K
+        self.local_fn = local_fn or self._library_local
+        self.merge_fn = merge_fn or self._library_merge
         dev = W2_shard.device
         R = B * K
         self.local = torch.empty(2, R, s, dtype=torch.int32, device=dev)
         self.gathered = torch.empty(self.G, 2, R, s, dtype=torch.int32, device=dev)
         self.v0_dev = torch.tensor(shard_offsets(V, self.G, align), dtype=torch.int32, device=dev)
-        self.ws = torch.empty(max(256, api.heads_workspace_size(B, W1.shape[1], Vr, K, s, W1.dtype)),
-                              dtype=torch.uint8, device=dev)
+        self.ws = (torch.empty(max(256, api.heads_workspace_size(B, W1.shape[1], Vr, K, s,
+                                                                 W1.dtype)),
+                               dtype=torch.uint8, device=dev) if local_fn is None else None)
         self.out = (torch.empty(B, K, s, dtype=torch.int32, device=dev),
                     torch.empty(B, K, s, dtype=torch.float32, device=dev))
+
+    def _library_local(self, h, W1, b1, W2, s, idx, val):
+        api.medusa_heads_forward(h, W1, b1, W2, s=s, want_logits=False, out=(None, idx, val),
+                                 ws=self.ws)
+
+    @staticmethod
+    def _library_merge(gathered, s, v0, out_idx, out_val):
+        api.medusa_topk_merge_planes(gathered, s, v0, out=(out_idx, out_val))
 
     def local_topk(self, h):
         """This rank's s best ids (local to its slice) and values per (b, k),
@@ -103,17 +120,16 @@ class ShardedHeads:
         B, K, s = self.B, self.K, self.s
         val = self.local[0].view(torch.float32).view(B, K, s)
         idx = self.local[1].view(B, K, s)
-        api.medusa_heads_forward(h, self.W1, self.b1, self.W2, s=s, want_logits=False,
-                                 out=(None, idx, val), ws=self.ws)
+        self.local_fn(h, self.W1, self.b1, self.W2, s, idx, val)
         return self.local
 
-    def __call__(self, h):
+    def __call__(self, h, out=None):
         """topk_idx [B][K][s] int32 (ids of the whole vocabulary) and
-        topk_val [B][K][s] fp32, the same on every rank."""
+        topk_val [B][K][s] fp32, the same on every rank (into `out` when
+        given)."""
         self.local_topk(h)
         gather_candidates(self.local, self.group, out=self.gathered)
         R = self.B * self.K
-        oi, ov = self.out
-        api.medusa_topk_merge_planes(self.gathered, self.s, self.v0_dev,
-                                     out=(oi.view(R, self.s), ov.view(R, self.s)))
+        oi, ov = self.out if out is None else out
+        self.merge_fn(self.gathered, self.s, self.v0_dev, oi.view(R, self.s), ov.view(R, self.s))
         return oi, ov

@@ -88,7 +88,10 @@ def test_validation_before_any_launch():
                                     1 << 20, None) == L.ERR_UNSUPPORTED
     assert lib.medusa_heads_forward(p, p, None, p, 1, 64, 10, 2, L.BF16, None, 1, None, None, p,
                                     1 << 20, None) == L.ERR_INVALID_ARG
-    assert lib.medusa_heads_forward(p, p, None, p, 33, 64, 10, 2, L.BF16, p, 1, p, None, p,
+    # bf16 batches beyond MEDUSA_MAX_HEADS_B (4096); fp32 beyond 16
+    assert lib.medusa_heads_forward(p, p, None, p, 4097, 64, 10, 2, L.BF16, p, 1, p, None, p,
+                                    1 << 20, None) == L.ERR_UNSUPPORTED
+    assert lib.medusa_heads_forward(p, p, None, p, 17, 64, 10, 2, L.F32, p, 1, p, None, p,
                                     1 << 20, None) == L.ERR_UNSUPPORTED
     assert lib.medusa_heads_forward(C.c_void_p(258), p, None, p, 1, 64, 10, 2, L.BF16, p, 1, p,
                                     None, p, 1 << 20, None) == L.ERR_INVALID_ARG
