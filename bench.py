@@ -375,17 +375,25 @@ def kernel_figures(cfg, st, calls, pk) -> dict:
     if cfg.accept in ("typical", "both"):
         out["accept_typical"] = KB.time_accept(cfg, st.vlogits, st.tree_tok, st.tree, calls,
                                                typical=True, ws=st.ws_acc, pk=pk)
-    # the bound that sets each kernel's floor: HBM bytes or tensor-core flops
     for r in out.values():
-        if "algorithmic_flops" in r:
-            t_hbm = r["algorithmic_bytes"] / (pk["hbm_gbs"] * 1e9)
-            t_tc = r["algorithmic_flops"] / (pk["bf16_tflops"] * 1e12)
-            r["bound"] = "tensor" if t_tc > t_hbm else "hbm"
-            r["floor_ms"] = 1e3 * max(t_hbm, t_tc)
-        else:
-            r["bound"] = "hbm"
-            r["floor_ms"] = 1e3 * r["algorithmic_bytes"] / (pk["hbm_gbs"] * 1e9)
+        classify(r, pk)
     return out
+
+
+def classify(r: dict, pk: dict) -> dict:
+    """Adds to a kernel figure the bound that sets its floor (HBM bytes or
+    tensor-core flops, whichever takes longer at the peaks), the floor time,
+    `frac` against the peak of that bound, `hbm_frac`, and `roofline_frac`
+    = floor time / measured time."""
+    hbm_frac = r["algorithmic_bytes"] / (r["avg_ms"] / 1e3) / 1e9 / pk["hbm_gbs"]
+    t_hbm = r["algorithmic_bytes"] / (pk["hbm_gbs"] * 1e9)
+    t_tc = r["algorithmic_flops"] / (pk["bf16_tflops"] * 1e12) if "algorithmic_flops" in r else 0.0
+    r["bound"] = "tensor" if t_tc > t_hbm else "hbm"
+    r["floor_ms"] = 1e3 * max(t_hbm, t_tc)
+    r["hbm_frac"] = hbm_frac
+    r["frac"] = r["tensor_frac"] if r["bound"] == "tensor" else hbm_frac
+    r["roofline_frac"] = r["floor_ms"] / r["avg_ms"]
+    return r
 
 
 def roofline_of(name: str, r: dict, pk: dict, workload: str) -> dict:
@@ -398,14 +406,15 @@ def roofline_of(name: str, r: dict, pk: dict, workload: str) -> dict:
     line = {"kernel": name, "bound": r["bound"], "achieved": ach, "peak": peak, "unit": unit,
             "frac": ach / peak, "traffic": traffic, "peak_src": pk["src"],
             "avg_ms": r["avg_ms"], "calls": r["calls"],
-            "algorithmic_bytes": r["algorithmic_bytes"],
+            "algorithmic_bytes": r["algorithmic_bytes"], "floor_ms": r.get("floor_ms"),
+            "roofline_frac": r.get("roofline_frac"),
             "timing": f"CUDA events around {r['calls']} back-to-back calls on the launching "
                       f"stream, after the timed steps"}
     if "algorithmic_flops" in r:
         line.update({"algorithmic_flops": r["algorithmic_flops"], "tflops": r["tflops"],
                      "tensor_frac": r["tensor_frac"],
                      "tensor_frac_sustained": r["tensor_frac_sustained"],
-                     "hbm_frac": r["frac"]})
+                     "hbm_frac": r["hbm_frac"]})
     if traffic:
         line["traffic_over_algorithmic"] = traffic / r["algorithmic_bytes"]
     return line
@@ -445,11 +454,12 @@ def other_workloads(args, headline, dev, rank, pk) -> dict:
         kern = kernel_figures(cfg, st, KERNEL_CALLS, pk)
         res[name] = {"steps_per_s": EXTRA_STEPS / t, "ms_per_step": 1e3 * t / EXTRA_STEPS,
                      "steps": EXTRA_STEPS, "dtype": cfg.dtype, "batch": cfg.B,
-                     "kernels": {k: {kk: v[kk] for kk in ("avg_ms", "achieved", "unit", "frac",
-                                                         "bound", "floor_ms", "tflops",
-                                                         "tensor_frac", "key_chunks",
-                                                         "query_tiles_per_cta") if kk in v}
-                                 for k, v in kern.items()}}
+                     "kernels": {k: dict({kk: v[kk] for kk in (
+                         "avg_ms", "achieved", "unit", "frac", "bound", "floor_ms",
+                         "roofline_frac", "hbm_frac", "tflops", "tensor_frac", "key_chunks",
+                         "query_tiles_per_cta") if kk in v},
+                         traffic=stored_traffic(name, k) if k in TRAFFIC_SOURCES else None)
+                         for k, v in kern.items()}}
         del st
         torch.cuda.empty_cache()
     return res
@@ -469,7 +479,7 @@ def heads_large_batch_figure(dev, pk) -> dict:
     name, B = LARGE_BATCH
     c = CONFIGS[name].scaled(B=B)
     x = gen_head_inputs(c, dev, 0)
-    r = KB.time_heads(c, x, 20, pk=pk)
+    r = classify(KB.time_heads(c, x, 20, pk=pk), pk)
     exe = 2 * c.B * c.K * c.d * c.d + 2 * (2 * c.B) * c.K * c.V * c.d
     r.update({"workload": f"{name} heads at B = {B}", "batch": B,
               "executed_flops": exe,

@@ -13,16 +13,30 @@ PK = {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0,
 
 
 def test_roofline_hbm_and_tensor_bound():
-    r = {"avg_ms": 1.0, "calls": 50, "algorithmic_bytes": 3.25e9, "achieved": 3250.0,
-         "frac": 0.5, "bound": "hbm", "algorithmic_flops": 8e11, "tflops": 800.0,
-         "tensor_frac": 0.5, "tensor_frac_sustained": 800 / 1400}
-    line = bench.roofline_of("tree_attention", r, PK, "no_such_workload")
+    # 3.25 GB in 1 ms against 6500 GB/s: HBM floor 0.5 ms; 8e11 flop against
+    # 1600 TF/s: tensor floor 0.5 ms (ties go to HBM)
+    pk = dict(PK, bf16_tflops=1600.0)
+    r = bench.classify({"avg_ms": 1.0, "calls": 50, "algorithmic_bytes": 3.25e9,
+                        "achieved": 3250.0, "algorithmic_flops": 8e11, "tflops": 800.0,
+                        "tensor_frac": 0.5, "tensor_frac_sustained": 800 / 1400}, pk)
+    assert r["bound"] == "hbm" and r["floor_ms"] == pytest.approx(0.5)
+    line = bench.roofline_of("tree_attention", r, pk, "no_such_workload")
     assert line["unit"] == "GB/s" and line["peak"] == 6500.0
     assert line["frac"] == pytest.approx(0.5) and line["traffic"] is None
-    r["bound"] = "tensor"
-    line = bench.roofline_of("tree_attention", r, PK, "no_such_workload")
-    assert line["unit"] == "TFLOP/s" and line["frac"] == pytest.approx(0.5)
-    assert line["hbm_frac"] == pytest.approx(0.5)
+    assert line["roofline_frac"] == pytest.approx(0.5)
+    # twice the flops: tensor-bound, floor 1.0 ms, frac against the bf16 peak
+    r = bench.classify({"avg_ms": 1.25, "calls": 50, "algorithmic_bytes": 3.25e9,
+                        "achieved": 2600.0, "algorithmic_flops": 1.6e12, "tflops": 1280.0,
+                        "tensor_frac": 0.8, "tensor_frac_sustained": 1280 / 1400}, pk)
+    assert r["bound"] == "tensor" and r["floor_ms"] == pytest.approx(1.0)
+    assert r["frac"] == pytest.approx(0.8) and r["hbm_frac"] == pytest.approx(0.4)
+    line = bench.roofline_of("tree_attention", r, pk, "no_such_workload")
+    assert line["unit"] == "TFLOP/s" and line["frac"] == pytest.approx(0.8)
+    assert line["hbm_frac"] == pytest.approx(0.4) and line["roofline_frac"] == pytest.approx(0.8)
+    # no flops: HBM-bound
+    r = bench.classify({"avg_ms": 2.0, "calls": 5, "algorithmic_bytes": 6.5e9,
+                        "achieved": 3250.0}, pk)
+    assert r["bound"] == "hbm" and r["frac"] == pytest.approx(0.5)
 
 
 def test_stored_traffic_goes_stale_when_sources_change(tmp_path):
