@@ -135,43 +135,34 @@ __device__ __forceinline__ void red_consume(RedState& st, const float (&x)[NV], 
     if (st.sf.m != -INFINITY) {  // else every value so far is -inf: nothing to add
       const unsigned long long zs2 = f2_pack(zscale, zscale);
       const unsigned long long nm2 = f2_pack(-st.sf.m, -st.sf.m);
-      if (NV == 1) {  // unaligned rows: one logit at a time, on lane 0
+      if constexpr (NV == 1) {  // unaligned rows: one logit at a time, on lane 0
         const float t = fmaxf(fmaf(x[0], zscale, -st.sf.m), -200.f);
         const float e = ex2_approx(t);
         st.Z2 = f2_add(st.Z2, f2_pack(e, 0.f));
         st.S2 = f2_fma(f2_pack(e, 0.f), f2_pack(t, 0.f), st.S2);
-        return;
-      }
+      } else {
 #pragma unroll
-      for (int j = 0; j + 1 < NV; j += 2) {
-        // t <= 0; clamped so that a -inf (or NaN) logit adds 0 to Z and S
-        float t0, t1;
-        f2_unpack(f2_fma(f2_pack(x[j], x[(j + 1) % NV]), zs2, nm2), t0, t1);
-        t0 = fmaxf(t0, -200.f);
-        t1 = fmaxf(t1, -200.f);
-        const unsigned long long e2 = f2_pack(ex2_approx(t0), ex2_approx(t1));
-        st.Z2 = f2_add(st.Z2, e2);
-        st.S2 = f2_fma(e2, f2_pack(t0, t1), st.S2);
+        for (int j = 0; j + 1 < NV; j += 2) {
+          // t <= 0; clamped so that a -inf (or NaN) logit adds 0 to Z and S
+          float t0, t1;
+          f2_unpack(f2_fma(f2_pack(x[j], x[j + 1]), zs2, nm2), t0, t1);
+          t0 = fmaxf(t0, -200.f);
+          t1 = fmaxf(t1, -200.f);
+          const unsigned long long e2 = f2_pack(ex2_approx(t0), ex2_approx(t1));
+          st.Z2 = f2_add(st.Z2, e2);
+          st.S2 = f2_fma(e2, f2_pack(t0, t1), st.S2);
+        }
       }
     }
   }
 }
 
+// Chunk sp of verify row `row` reduced by one CTA: the argmax key and, with
+// TYPICAL, the softmax statistics at scale zscale.
 template <typename T, bool TYPICAL>
-__global__ void __launch_bounds__(kRedThreads)
-    row_reduce_kernel(const T* __restrict__ vlog, int V, int chunk, int splits, ZTab zt,
-                      const int32_t* __restrict__ depth, int N, int K,
-                      RowPart* __restrict__ parts) {
-  // nothing in this kernel runs ahead of its predecessor
-  griddep_launch_dependents();
-  griddep_wait();
-  const size_t row = blockIdx.x;
-  float zscale = 0.f;
-  if (TYPICAL) {
-    const int dc = depth[row % (size_t)N] + 1;
-    zscale = zt.z[dc < K ? dc : K];
-  }
-  const int sp = blockIdx.y;
+__device__ __forceinline__ void row_reduce_chunk(const T* __restrict__ vlog, int V, int chunk,
+                                                 int splits, float zscale, size_t row, int sp,
+                                                 RowPart* __restrict__ parts) {
   const int lo = sp * chunk;
   const int hi = min(V, lo + chunk);
   const T* xr = vlog + row * (size_t)V;
@@ -252,6 +243,31 @@ __global__ void __launch_bounds__(kRedThreads)
     rp.pad = 0.f;
     parts[row * splits + sp] = rp;
   }
+}
+
+// Typical acceptance tests a node against its parent's row only, so the
+// softmax statistics are needed for the rows of nodes that have children;
+// a leaf's row is reduced to its argmax alone (the next token when that
+// leaf ends the accepted path) and reports (m, Z, S) = (-inf, 0, 0).
+template <typename T, bool TYPICAL>
+__global__ void __launch_bounds__(kRedThreads)
+    row_reduce_kernel(const T* __restrict__ vlog, int V, int chunk, int splits, ZTab zt,
+                      const int32_t* __restrict__ depth, const int32_t* __restrict__ nchild,
+                      int N, int K, RowPart* __restrict__ parts) {
+  // nothing in this kernel runs ahead of its predecessor
+  griddep_launch_dependents();
+  griddep_wait();
+  const size_t row = blockIdx.x;
+  const int sp = blockIdx.y;
+  if (TYPICAL) {
+    const int node = (int)(row % (size_t)N);
+    if (nchild[node] > 0) {  // CTA-uniform
+      const int dc = depth[node] + 1;
+      row_reduce_chunk<T, true>(vlog, V, chunk, splits, zt.z[dc < K ? dc : K], row, sp, parts);
+      return;
+    }
+  }
+  row_reduce_chunk<T, false>(vlog, V, chunk, splits, 0.f, row, sp, parts);
 }
 
 // One CTA per sequence, one thread per tree node (blockDim = N rounded up to
@@ -401,7 +417,7 @@ int accept_launch(const AcceptArgs& a, cudaStream_t st) {
 #define MEDUSA_ACC(T, TYP)                                                                     \
   do {                                                                                         \
     le = launch_pdl(row_reduce_kernel<T, TYP>, g1, dim3(kRedThreads), 0, st, (const T*)a.vlog, \
-                    a.V, P.chunk, P.splits, zt, t->d_depth, N, t->K, parts);                   \
+                    a.V, P.chunk, P.splits, zt, t->d_depth, t->d_nchild, N, t->K, parts);    \
     if (le == cudaSuccess)                                                                     \
       le = launch_pdl(accept_walk_kernel<T, TYP>, dim3(a.B), dim3(walk_threads), 0, st,        \
                       (const T*)a.vlog, parts, P.splits, a.tok, t->d_parent, t->d_depth,       \
@@ -511,7 +527,7 @@ int accept_greedy_noalloc_launch(const void* vlog, int dtype, const int32_t* tok
 #define MEDUSA_ACC_STATIC(T)                                                                     \
   do {                                                                                           \
     le = launch_pdl(row_reduce_kernel<T, false>, g1, dim3(kRedThreads), 0, st, (const T*)vlog, V, \
-                    P.chunk, P.splits, zt0, t->d_depth, N, t->K, parts);                         \
+                    P.chunk, P.splits, zt0, t->d_depth, t->d_nchild, N, t->K, parts);            \
     if (le == cudaSuccess)                                                                       \
       le = launch_pdl(accept_walk_kernel<T, false>, dim3(B), dim3(walk_threads), 0, st,          \
                       (const T*)vlog,                                                            \

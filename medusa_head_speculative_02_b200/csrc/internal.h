@@ -15,12 +15,14 @@ struct medusa_tree {
   int K = 0, s = 0, N = 0, W = 0;  // W = 32-bit words per ancestor-mask row
   int device = -1;
   std::vector<int32_t> parent, depth, rank_path, head_rank;
+  std::vector<int32_t> nchild;  // children of every node (0: a leaf)
   std::vector<uint32_t> anc;
   // device copies (one allocation owned by the plan)
   void* d_block = nullptr;
   const int32_t* d_parent = nullptr;
   const int32_t* d_depth = nullptr;
   const int32_t* d_head_rank = nullptr;  // (D-1)*s + r_D, -1 for the root
+  const int32_t* d_nchild = nullptr;
   const uint32_t* d_anc = nullptr;
 };
 

@@ -313,8 +313,10 @@ int medusa_tree_create(int K, int s, int N, medusa_tree_t** out) {
       delete t;
       return cuda_fail(e, "cudaGetDevice");
     }
+    t->nchild.assign(N, 0);
+    for (int c = 1; c < N; ++c) t->nchild[t->parent[c]]++;
     const size_t n4 = (size_t)N * 4;
-    const size_t bytes = 3 * n4 + (size_t)N * t->W * 4;
+    const size_t bytes = 4 * n4 + (size_t)N * t->W * 4;
     e = cudaMalloc(&t->d_block, bytes);
     if (e != cudaSuccess) {
       delete t;
@@ -324,7 +326,8 @@ int medusa_tree_create(int K, int s, int N, medusa_tree_t** out) {
     memcpy(host.data(), t->parent.data(), n4);
     memcpy(host.data() + n4, t->depth.data(), n4);
     memcpy(host.data() + 2 * n4, t->head_rank.data(), n4);
-    memcpy(host.data() + 3 * n4, t->anc.data(), (size_t)N * t->W * 4);
+    memcpy(host.data() + 3 * n4, t->nchild.data(), n4);
+    memcpy(host.data() + 4 * n4, t->anc.data(), (size_t)N * t->W * 4);
     e = cudaMemcpy(t->d_block, host.data(), bytes, cudaMemcpyHostToDevice);
     if (e != cudaSuccess) {
       cudaFree(t->d_block);
@@ -335,7 +338,8 @@ int medusa_tree_create(int K, int s, int N, medusa_tree_t** out) {
     t->d_parent = (const int32_t*)d;
     t->d_depth = (const int32_t*)(d + n4);
     t->d_head_rank = (const int32_t*)(d + 2 * n4);
-    t->d_anc = (const uint32_t*)(d + 3 * n4);
+    t->d_nchild = (const int32_t*)(d + 3 * n4);
+    t->d_anc = (const uint32_t*)(d + 4 * n4);
     *out = t;
     return MEDUSA_OK;
   } catch (...) {
