@@ -257,7 +257,12 @@ __global__ void __launch_bounds__(kRedThreads)
   // nothing in this kernel runs ahead of its predecessor
   griddep_launch_dependents();
   griddep_wait();
-  const size_t row = blockIdx.x;
+  // typical: rows taken node-major (node 0 of every sequence, then node 1,
+  // ...): the nodes with children, whose rows cost the exponentials, come
+  // first in (depth, lexicographic) order, so the launch ends on cheap rows
+  const unsigned nseq = gridDim.x / (unsigned)N;
+  const size_t row = TYPICAL ? (size_t)(blockIdx.x % nseq) * N + blockIdx.x / nseq
+                             : (size_t)blockIdx.x;
   const int sp = blockIdx.y;
   if (TYPICAL) {
     const int node = (int)(row % (size_t)N);
