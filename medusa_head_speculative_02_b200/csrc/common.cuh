@@ -421,8 +421,11 @@ __device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsig
 // obtained by adding 1.5 * 2^23, and f in [-0.5, 0.5]; 2^f by the degree-3
 // polynomial that minimises the maximum relative error on [-0.5, 0.5]
 // (coefficients fitted by Remez exchange: max relative error 7.5e-5,
-// 1.5e-4 once evaluated in fp32); 2^n by adding n to the exponent field.
-// For x <= 127; x < -126 gives 2^-126.
+// 1.5e-4 once evaluated in fp32); 2^n by adding n to the exponent field:
+// the bits of t = 1.5 * 2^23 + n shifted left by 23 are n << 23 modulo 2^32
+// (the low 9 bits of 1.5 * 2^23's bit pattern are zero), so one integer
+// multiply-add per lane forms the result.  For x <= 127; x < -126 gives
+// 2^-126.
 constexpr float kExp2C0 = 0.99992805719f;
 constexpr float kExp2C1 = 0.69326096773f;
 constexpr float kExp2C2 = 0.24261112511f;
@@ -430,8 +433,9 @@ constexpr float kExp2C3 = 0.05517166853f;
 __device__ __forceinline__ void exp2_fma2(float x0, float x1, float& e0, float& e1) {
   const unsigned long long x2 = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
   const unsigned long long t2 = f2_add(x2, f2_pack(12582912.0f, 12582912.0f));
-  const unsigned long long f2 = f2_add(x2, f2_add(t2, f2_pack(-12582912.0f, -12582912.0f)) ^
-                                               0x8000000080000000ull);
+  unsigned long long r2, f2;  // r = round(x), f = x - r
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r2) : "l"(t2), "l"(f2_pack(12582912.0f, 12582912.0f)));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f2) : "l"(x2), "l"(r2));
   const unsigned long long p2 =
       f2_fma(f2_fma(f2_fma(f2_pack(kExp2C3, kExp2C3), f2, f2_pack(kExp2C2, kExp2C2)), f2,
                     f2_pack(kExp2C1, kExp2C1)),
@@ -439,8 +443,11 @@ __device__ __forceinline__ void exp2_fma2(float x0, float x1, float& e0, float& 
   float t0, t1, p0, p1;
   f2_unpack(t2, t0, t1);
   f2_unpack(p2, p0, p1);
-  e0 = __int_as_float(__float_as_int(p0) + ((__float_as_int(t0) - 0x4B400000) << 23));
-  e1 = __int_as_float(__float_as_int(p1) + ((__float_as_int(t1) - 0x4B400000) << 23));
+  uint32_t u0, u1;
+  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(u0) : "r"(__float_as_uint(t0)), "r"(__float_as_uint(p0)));
+  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(u1) : "r"(__float_as_uint(t1)), "r"(__float_as_uint(p1)));
+  e0 = __uint_as_float(u0);
+  e1 = __uint_as_float(u1);
 }
 // Hardware base-2 exponential (MUFU ex2, approximate, flush-to-zero); used
 // where a few ulp are far below the bf16 rounding that follows.

@@ -21,16 +21,33 @@ def _coeffs():
     return c[0], c[1], c[2], c[3]
 
 
-def _exp2_fma(x):
+def _poly_parts(x):
     x = np.maximum(np.float32(x), np.float32(-126.0)).astype(np.float32)
     c0, c1, c2, c3 = _coeffs()
     t = (x + np.float32(12582912.0)).astype(np.float32)
-    n = t.view(np.int32) - np.int32(0x4B400000)
     f = (x - (t - np.float32(12582912.0)).astype(np.float32)).astype(np.float32)
     p = np.float32(c3)
     for c in (c2, c1, c0):            # fp32 fused multiply-add per step
         p = (p.astype(np.float64) * f + c).astype(np.float32)
-    return (p.view(np.int32) + (n << 23)).view(np.float32)
+    return np.atleast_1d(t), np.atleast_1d(p)
+
+
+def _exp2_fma(x):
+    """As the kernel forms it: one integer multiply-add per lane, the bits
+    of t times 2^23 plus the bits of p, modulo 2^32."""
+    t, p = _poly_parts(x)
+    u = (p.view(np.uint32).astype(np.uint64) + t.view(np.uint32).astype(np.uint64) * (1 << 23))
+    return (u & 0xFFFFFFFF).astype(np.uint32).view(np.float32)
+
+
+def test_exponent_insertion_equals_adding_n_to_the_exponent_field():
+    # n = bits(t) - bits(1.5 * 2^23) = round(x); p * 2^n by adding n << 23
+    x = np.linspace(-126.0, 9.0, 200001).astype(np.float32)
+    t, p = _poly_parts(x)
+    n = t.view(np.int32) - np.int32(0x4B400000)
+    assert np.array_equal(n, np.rint(np.maximum(x, -126.0)).astype(np.int32))
+    direct = (p.view(np.int32) + (n << 23)).view(np.float32)
+    assert np.array_equal(_exp2_fma(x).view(np.uint32), direct.view(np.uint32))
 
 
 def test_exp2_fma_relative_error_bound():
