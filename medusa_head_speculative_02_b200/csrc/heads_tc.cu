@@ -350,21 +350,20 @@ __global__ void heads_silu_kernel(const float* __restrict__ part, int S, int K, 
                                   int ncnt2) {
   griddep_launch_dependents();  // stage 2 may start streaming its weights
   griddep_wait();
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  for (int j = i; j < ncnt2; j += gridDim.x * blockDim.x) cnt2[j] = 0;
-  if (i >= K * d) return;
-  const int kh = i / d, m = i - kh * d;
-  const float bias = b1 ? __bfloat162float(b1[i]) : 0.f;
-  for (int b = 0; b < B; ++b) {
-    float a = bias;
-    for (int s2 = 0; s2 < S; ++s2) a += part[(((size_t)s2 * K + kh) * B + b) * d + m];
-    const float uu = a / (1.f + expf(-a)) + __bfloat162float(h[(size_t)b * d + m]);
-    const __nv_bfloat16 hi = __float2bfloat16_rn(uu);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(uu - __bfloat162float(hi));
-    __nv_bfloat16* urow = u + ((size_t)kh * 2 * B + 2 * b) * d + m;
-    urow[0] = hi;
-    urow[d] = lo;
-  }
+  // one thread per (head, sequence, feature): i = (kh * B + b) * d + m
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  for (long long j = i; j < ncnt2; j += (long long)gridDim.x * blockDim.x) cnt2[j] = 0;
+  if (i >= (long long)K * B * d) return;
+  const int m = (int)(i % d);
+  const int kb = (int)(i / d), kh = kb / B, b = kb - kh * B;
+  float a = b1 ? __bfloat162float(b1[(size_t)kh * d + m]) : 0.f;
+  for (int s2 = 0; s2 < S; ++s2) a += part[(((size_t)s2 * K + kh) * B + b) * d + m];
+  const float uu = a / (1.f + expf(-a)) + __bfloat162float(h[(size_t)b * d + m]);
+  const __nv_bfloat16 hi = __float2bfloat16_rn(uu);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(uu - __bfloat162float(hi));
+  __nv_bfloat16* urow = u + ((size_t)kh * 2 * B + 2 * b) * d + m;
+  urow[0] = hi;
+  urow[d] = lo;
 }
 
 int choose_splits(int tiles, int kchunks, int sms, double want) {
@@ -494,8 +493,9 @@ int heads_tc_launch(const HeadsArgs& a, cudaStream_t st) {
   int rc = dispatch_stage(P.nc1, mA1, mB1, p1, st);
   if (rc) return rc;
   {
-    const int n = a.K * a.d;
-    cudaError_t e2 = launch_pdl(heads_silu_kernel, dim3((n + 255) / 256), dim3(256), 0, st, p1.part,
+    const long long n = (long long)a.K * a.B * a.d;
+    cudaError_t e2 = launch_pdl(heads_silu_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0,
+                                st, p1.part,
                                 P.S1, a.K, a.B, a.d, (const __nv_bfloat16*)a.b1,
                                 (const __nv_bfloat16*)a.h, u, counters + (size_t)a.K * P.mt1,
                                 a.K * P.mt2);
