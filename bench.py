@@ -324,7 +324,9 @@ def run_reference(args, cfg, world, rank):
                        "accept": cfg.accept},
             "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores, "kind": "oracle",
                              "sample": S.sample_desc(), "wall_s": wall,
-                             "setup_s": t0 - t_setup},
+                             "setup_s": t0 - t_setup,
+                             "method": "extrapolated: each operation timed on a slice of its "
+                                       "rows and scaled to the whole step"},
             "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
