@@ -557,8 +557,8 @@ def run_tensor_parallel(args, cfg, world, rank, local):
     time.sleep(0.3)
     elapsed_s = time_steps(st, K, dev)
     t = max_over_ranks(elapsed_s, dev)
-    attn = KB.time_attention(lcfg, st.x, st.tree, KERNEL_CALLS, ws=st.ws_attn, pk=pk)
-    heads = KB.time_heads(lcfg.scaled(V=v1 - v0), st.x, KERNEL_CALLS, pk=pk)
+    attn = classify(KB.time_attention(lcfg, st.x, st.tree, KERNEL_CALLS, ws=st.ws_attn, pk=pk), pk)
+    heads = classify(KB.time_heads(lcfg.scaled(V=v1 - v0), st.x, KERNEL_CALLS, pk=pk), pk)
     clk = clocks.stop()
     if rank == 0:
         line = {"metric": METRIC, "value": K / t, "unit": "steps/s", "n_gpus": world, "steps": K,
@@ -816,19 +816,32 @@ def main(argv=None):
     world, rank, local = dist_env()
     if args.impl == "reference":
         return run_reference(args, cfg, world, rank)
-    if world > 1:
+    # vocab-shard needs a process group even on one rank (G = 1: the whole
+    # vocabulary on one GPU, the all-gather a copy)
+    use_pg = world > 1 or args.heads == "vocab-shard"
+    if use_pg:
         import datetime
+        if world == 1:
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", str(_free_port()))
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
     try:
         if args.heads == "vocab-shard":
-            if world < 2:
-                raise SystemExit("--heads vocab-shard needs torchrun with 2 or more ranks")
             return run_tensor_parallel(args, cfg, world, rank, local)
         return run_ours(args, cfg, world, rank, local)
     finally:
-        if world > 1:
+        if use_pg:
             torch.distributed.destroy_process_group()
+
+
+def _free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
 
 
 if __name__ == "__main__":
