@@ -289,6 +289,24 @@ int medusa_accept_typical(const void* vlogits, int dtype,
                           size_t ws_bytes, void* stream);
 
 /*
+ * Greedy and typical acceptance of the same verify logits in one pass over
+ * them (a workload that verifies under both rules, as the long-context
+ * configuration does): writes exactly what medusa_accept_greedy (g_*) and
+ * medusa_accept_typical (t_*) write for the same arguments.  One row
+ * reduction serves both walks, since the typical pass keeps every row's
+ * argmax.  Workspace: medusa_accept_workspace_size's.  The two output sets
+ * must not overlap.
+ */
+int medusa_accept_greedy_typical(const void* vlogits, int dtype,
+                                 const int32_t* tree_tok,
+                                 const medusa_tree_t* tree, int B, int V,
+                                 float temperature, float eps, float delta,
+                                 int32_t* g_accept_len, int32_t* g_accept_nodes,
+                                 int32_t* g_next_tok, int32_t* t_accept_len,
+                                 int32_t* t_accept_nodes, int32_t* t_next_tok,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Typical acceptance with one temperature per head.  [ZH] "4.2 温度调优"
  * tunes a temperature per Medusa head; reading: head D proposes the
  * candidates of depth D, and each is verified on its parent's row at

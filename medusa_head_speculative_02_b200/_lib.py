@@ -48,6 +48,8 @@ SIGNATURES = {
     "medusa_accept_workspace_size": (csz, [vp, ci, ci]),
     "medusa_accept_greedy": (ci, [vp, ci, vp, vp, ci, ci, vp, vp, vp, vp, csz, vp]),
     "medusa_accept_typical": (ci, [vp, ci, vp, vp, ci, ci, cf, cf, cf, vp, vp, vp, vp, csz, vp]),
+    "medusa_accept_greedy_typical": (ci, [vp, ci, vp, vp, ci, ci, cf, cf, cf, vp, vp, vp, vp, vp,
+                                          vp, vp, csz, vp]),
     "medusa_accept_typical_per_head": (ci, [vp, ci, vp, vp, ci, ci, f32p, cf, cf, vp, vp, vp, vp,
                                             csz, vp]),
     "medusa_accept_greedy_noalloc": (ci, [vp, ci, vp, vp, ci, ci, vp, vp, vp, vp]),

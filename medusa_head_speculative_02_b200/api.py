@@ -292,6 +292,27 @@ def medusa_accept_typical(vlogits, tree_tok, tree: Tree, temperature: float, eps
     return alen, anodes, nxt
 
 
+def medusa_accept_greedy_typical(vlogits, tree_tok, tree: Tree, temperature: float,
+                                 eps: float = 0.09, delta: float = 0.6, out_greedy=None,
+                                 out_typical=None, ws=None):
+    """Greedy and typical acceptance of the same verify logits from one pass
+    over them; returns ((accept_len, accept_nodes, next_tok) greedy,
+    (accept_len, accept_nodes, next_tok) typical)."""
+    B, N, V = vlogits.shape
+    _need(vlogits, "vlogits")
+    _need(tree_tok, "tree_tok", torch.int32, (B, N))
+    g = out_greedy if out_greedy is not None else _accept_outputs(B, tree.K, vlogits.device)
+    t = out_typical if out_typical is not None else _accept_outputs(B, tree.K, vlogits.device)
+    need = accept_workspace_size(tree, B, V)
+    if ws is None or ws.numel() < need:
+        ws = _ws(need, vlogits.device)
+    L.check(L.lib().medusa_accept_greedy_typical(
+        _ptr(vlogits), _dt(vlogits), _ptr(tree_tok), tree.handle, B, V, float(temperature),
+        float(eps), float(delta), _ptr(g[0]), _ptr(g[1]), _ptr(g[2]), _ptr(t[0]), _ptr(t[1]),
+        _ptr(t[2]), _ptr(ws), ws.numel(), _stream(vlogits.device)), "medusa_accept_greedy_typical")
+    return g, t
+
+
 def medusa_accept_typical_per_head(vlogits, tree_tok, tree: Tree, temperatures, eps: float = 0.09,
                                    delta: float = 0.6, out=None, ws=None):
     """Typical acceptance with one temperature per head (the candidates of

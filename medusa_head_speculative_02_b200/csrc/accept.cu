@@ -429,13 +429,26 @@ int accept_launch(const AcceptArgs& a, cudaStream_t st) {
                       t->d_anc, N, t->W, t->K, a.V, zt, a.eps, a.delta, a.accept_len,          \
                       a.accept_nodes, a.next_tok);                                             \
   } while (0)
+  // greedy results from the typical pass's row reduction (its keys hold
+  // every row's argmax)
+#define MEDUSA_ACC_GREEDY(T)                                                                     \
+  do {                                                                                           \
+    if (le == cudaSuccess && a.typical && a.g_accept_len)                                        \
+      le = launch_pdl(accept_walk_kernel<T, false>, dim3(a.B), dim3(walk_threads), 0, st,        \
+                      (const T*)a.vlog, parts, P.splits, a.tok, t->d_parent, t->d_depth,         \
+                      t->d_anc, N, t->W, t->K, a.V, zt, 0.f, 0.f, a.g_accept_len,                \
+                      a.g_accept_nodes, a.g_next_tok);                                           \
+  } while (0)
   if (a.dtype == MEDUSA_F32) {
     if (a.typical) MEDUSA_ACC(float, true);
     else MEDUSA_ACC(float, false);
+    MEDUSA_ACC_GREEDY(float);
   } else {
     if (a.typical) MEDUSA_ACC(__nv_bfloat16, true);
     else MEDUSA_ACC(__nv_bfloat16, false);
+    MEDUSA_ACC_GREEDY(__nv_bfloat16);
   }
+#undef MEDUSA_ACC_GREEDY
 #undef MEDUSA_ACC
   cudaError_t e = le != cudaSuccess ? le : cudaGetLastError();
   return e == cudaSuccess ? MEDUSA_OK : cuda_fail(e, "accept kernels launch");

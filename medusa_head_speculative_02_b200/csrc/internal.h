@@ -170,6 +170,11 @@ struct AcceptArgs {
   int32_t* accept_len;
   int32_t* accept_nodes;
   int32_t* next_tok;
+  // typical only: also the greedy results from the same row reduction
+  // (null: none)
+  int32_t* g_accept_len = nullptr;
+  int32_t* g_accept_nodes = nullptr;
+  int32_t* g_next_tok = nullptr;
   void* ws;
   size_t ws_bytes;
 };

@@ -496,7 +496,8 @@ static int accept_common(const void* vlogits, int dtype, const int32_t* tree_tok
                          const medusa_tree_t* tree, int B, int V, bool typical, float T,
                          const float* temps, float eps, float delta, int32_t* accept_len,
                          int32_t* accept_nodes, int32_t* next_tok, void* ws, size_t ws_bytes,
-                         void* stream) {
+                         void* stream, int32_t* g_accept_len = nullptr,
+                         int32_t* g_accept_nodes = nullptr, int32_t* g_next_tok = nullptr) {
   int rc = check_tree(tree);
   if (rc) return rc;
   if (!dtype_ok(dtype)) return fail(MEDUSA_ERR_INVALID_ARG, "bad dtype");
@@ -529,6 +530,9 @@ static int accept_common(const void* vlogits, int dtype, const int32_t* tree_tok
   a.accept_len = accept_len;
   a.accept_nodes = accept_nodes;
   a.next_tok = next_tok;
+  a.g_accept_len = g_accept_len;
+  a.g_accept_nodes = g_accept_nodes;
+  a.g_next_tok = g_next_tok;
   a.ws = ws;
   a.ws_bytes = ws_bytes;
   return accept_launch(a, (cudaStream_t)stream);
@@ -550,6 +554,23 @@ int medusa_accept_typical(const void* vlogits, int dtype, const int32_t* tree_to
   medusa::NvtxRange nvtx_range("medusa_accept_typical");
   return accept_common(vlogits, dtype, tree_tok, tree, B, V, true, temperature, nullptr, eps,
                        delta, accept_len, accept_nodes, next_tok, ws, ws_bytes, stream);
+}
+
+int medusa_accept_greedy_typical(const void* vlogits, int dtype, const int32_t* tree_tok,
+                                 const medusa_tree_t* tree, int B, int V, float temperature,
+                                 float eps, float delta, int32_t* g_accept_len,
+                                 int32_t* g_accept_nodes, int32_t* g_next_tok,
+                                 int32_t* t_accept_len, int32_t* t_accept_nodes,
+                                 int32_t* t_next_tok, void* ws, size_t ws_bytes, void* stream) {
+  medusa::NvtxRange nvtx_range("medusa_accept_greedy_typical");
+  if (B > 0 && (!g_accept_len || !g_accept_nodes || !g_next_tok))
+    return fail(MEDUSA_ERR_INVALID_ARG, "NULL pointer");
+  if (B > 0 && (g_accept_len == t_accept_len || g_accept_nodes == t_accept_nodes ||
+                g_next_tok == t_next_tok))
+    return fail(MEDUSA_ERR_INVALID_ARG, "greedy and typical outputs overlap");
+  return accept_common(vlogits, dtype, tree_tok, tree, B, V, true, temperature, nullptr, eps,
+                       delta, t_accept_len, t_accept_nodes, t_next_tok, ws, ws_bytes, stream,
+                       g_accept_len, g_accept_nodes, g_next_tok);
 }
 
 int medusa_accept_typical_per_head(const void* vlogits, int dtype, const int32_t* tree_tok,

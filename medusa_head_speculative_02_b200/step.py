@@ -74,6 +74,12 @@ class VerifyStep:
 
     def accept(self):
         cfg = self.cfg
+        if cfg.accept == "both":  # one pass over the verify logits serves both rules
+            api.medusa_accept_greedy_typical(
+                self.vlogits, self.tree_tok, self.tree, cfg.temperature, cfg.eps, cfg.delta,
+                out_greedy=(self.accept_len, self.accept_nodes, self.next_tok),
+                out_typical=(self.accept_len2, self.accept_nodes2, self.next_tok2), ws=self.ws_acc)
+            return
         if cfg.accept in ("greedy", "both"):
             api.medusa_accept_greedy(self.vlogits, self.tree_tok, self.tree,
                                      out=(self.accept_len, self.accept_nodes, self.next_tok),
@@ -98,10 +104,10 @@ class VerifyStep:
 
     def launches_per_step(self) -> int:
         c = self.cfg
-        n_acc = 2 if c.accept == "both" else 1
+        # both rules: one row reduction and two walks
+        acc = LAUNCHES["accept"] + 1 if c.accept == "both" else LAUNCHES["accept"]
         attn = api.attention_launches(self.tree, c.B, c.Hq, c.Hkv, c.dh, c.Lcap, c.torch_dtype)
-        return (LAUNCHES["heads"] + LAUNCHES["build_tree"] + attn + n_acc * LAUNCHES["accept"] +
-                LAUNCHES["kv_compact"])
+        return (LAUNCHES["heads"] + LAUNCHES["build_tree"] + attn + acc + LAUNCHES["kv_compact"])
 
     # algorithmic work ---------------------------------------------------------
     def heads_bytes(self) -> int:
@@ -163,9 +169,9 @@ class MultiLayerStep:
     def launches_per_step(self) -> int:
         c = self.st.cfg
         attn = api.attention_launches(self.st.tree, c.B, c.Hq, c.Hkv, c.dh, c.Lcap, c.torch_dtype)
-        n_acc = 2 if c.accept == "both" else 1
-        return (LAUNCHES["heads"] + LAUNCHES["build_tree"] + self.layers * attn +
-                n_acc * LAUNCHES["accept"] + LAUNCHES["kv_compact"])
+        acc = LAUNCHES["accept"] + 1 if c.accept == "both" else LAUNCHES["accept"]
+        return (LAUNCHES["heads"] + LAUNCHES["build_tree"] + self.layers * attn + acc +
+                LAUNCHES["kv_compact"])
 
 
 class HostIO:

@@ -288,3 +288,32 @@ def test_kv_compact_exact(dtype, Hkv, dh):
 
 def test_device_status_clean():
     assert api.device_status(clear=True) == 0
+
+
+@pytest.mark.parametrize("B,K,s,N,V,dtype,T", [
+    (4, 5, 3, 256, 32000, "bf16", 0.7),
+    (3, 5, 10, 64, 1000, "bf16", 1.3),
+    (2, 4, 3, 16, 1024, "f32", 0.5),
+])
+def test_accept_greedy_typical_in_one_pass_equals_the_two_calls(B, K, s, N, V, dtype, T):
+    """medusa_accept_greedy_typical writes what medusa_accept_greedy and
+    medusa_accept_typical write for the same arguments, bit for bit, and the
+    greedy half equals the oracle's sequential argmax decoding."""
+    cfg = MedusaConfig("both", dtype, B=B, d=8, V=V, K=K, s=s, N=N, Hq=1, Hkv=1, dh=64,
+                       L_lo=0, L_hi=0)
+    plan = O.tree_plan(K, s, N)
+    g = torch.Generator().manual_seed(B * N + V)
+    topk = torch.stack([torch.randperm(V, generator=g)[:K * s].view(K, s) for _ in range(B)])
+    tok, _ = O.build_tree(plan, torch.randint(0, V, (B,), generator=g), topk, [0] * B)
+    vlog = plant_verify_logits(cfg, plan["parent"], tok, device=DEV, seed=B + K)
+    tok_d = torch.as_tensor(tok, dtype=torch.int32, device=DEV)
+    tree = api.Tree(K, s, N)
+    rg = api.medusa_accept_greedy(vlog, tok_d, tree)
+    rt = api.medusa_accept_typical(vlog, tok_d, tree, T)
+    fg, ft = api.medusa_accept_greedy_typical(vlog, tok_d, tree, T)
+    torch.cuda.synchronize()
+    for a, b in zip(fg + ft, rg + rt):
+        assert torch.equal(a, b)
+    ref = O.accept_greedy(vlog, tok, plan)
+    assert (fg[0].cpu().numpy() == ref[0]).all()
+    assert api.device_status() == 0

@@ -98,6 +98,13 @@ def test_validation_before_any_launch():
     assert lib.medusa_heads_forward(p, p, None, p, 1, 64, 10, 2, L.BF16, p, 11, p, None, p,
                                     1 << 20, None) == L.ERR_INVALID_ARG      # s > V
     assert lib.medusa_topk(p, L.BF16, 4, 10, 0, p, None, None) == L.ERR_INVALID_ARG
+    # both acceptance rules in one pass: greedy outputs missing, or shared with typical's
+    q, r = C.c_void_p(512), C.c_void_p(768)
+    assert lib.medusa_accept_greedy_typical(p, L.BF16, p, p, 2, 10, 0.7, 0.09, 0.6, None, q, r,
+                                            p, q, r, p, 1 << 20, None) == L.ERR_INVALID_ARG
+    assert lib.medusa_accept_greedy_typical(p, L.BF16, p, p, 2, 10, 0.7, 0.09, 0.6, p, q, r,
+                                            p, q, r, p, 1 << 20, None) == L.ERR_INVALID_ARG
+    assert b"overlap" in lib.medusa_last_error()
     assert lib.medusa_topk(p, L.BF16, 4, 10, 17, p, None, None) == L.ERR_INVALID_ARG
     # calls taking a tree reject a NULL plan
     assert lib.medusa_build_tree(None, p, p, p, 1, p, p, None) == L.ERR_INVALID_ARG
