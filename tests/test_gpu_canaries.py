@@ -10,7 +10,8 @@ written, no written float is NaN, and each output equals, bit for bit, the
 same call made on freshly allocated buffers.  The chain is the verify step
 of the Medusa paper digest ([MD] "ツリーアテンションによる並列検証"): heads +
 top-s, tree expansion, tree attention, acceptance, next-token sampling,
-compaction, plus the shard merge.
+compaction (both acceptance rules separately and in one pass), plus the
+shard merge.
 """
 import ctypes as C
 import math
@@ -144,6 +145,18 @@ def test_step_calls_stay_inside_their_buffers(case):
             _filled(q)
             assert torch.equal(q.t, rr)
         accepted = accepted or r
+    # both rules from one pass: two guarded output sets
+    rg = api.medusa_accept_greedy(vlog, rtok, tree)
+    rt = api.medusa_accept_typical(vlog, rtok, tree, 0.7)
+    gg = tuple(Guarded(x.shape, I32, DEV) for x in rg)
+    gt2 = tuple(Guarded(x.shape, I32, DEV) for x in rt)
+    api.medusa_accept_greedy_typical(vlog, rtok, tree, 0.7, out_greedy=tuple(q.t for q in gg),
+                                     out_typical=tuple(q.t for q in gt2), ws=wsc.t)
+    torch.cuda.synchronize()
+    assert wsc.intact()
+    for q, rr in zip(gg + gt2, rg + rt):
+        _filled(q)
+        assert torch.equal(q.t, rr)
     alen, anodes, _ = accepted
     for temp in (0.0, 0.8):
         rn = api.medusa_sample_next(vlog, alen, anodes, temp, seed=5, offset=1)
