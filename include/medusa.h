@@ -294,8 +294,9 @@ int medusa_accept_typical(const void* vlogits, int dtype,
  * configuration does): writes exactly what medusa_accept_greedy (g_*) and
  * medusa_accept_typical (t_*) write for the same arguments.  One row
  * reduction serves both walks, since the typical pass keeps every row's
- * argmax.  Workspace: medusa_accept_workspace_size's.  The two output sets
- * must not overlap.
+ * argmax.  Workspace: medusa_accept_workspace_size's.  Errors: those of
+ * medusa_accept_typical, and MEDUSA_ERR_INVALID_ARG (nothing launched) when
+ * a greedy output is NULL or the two output sets share a pointer.
  */
 int medusa_accept_greedy_typical(const void* vlogits, int dtype,
                                  const int32_t* tree_tok,
