@@ -1,6 +1,8 @@
 """CPU: host-side logic of bench.py's measurement lines (roofline object,
-stored DRAM traffic and its staleness check, per-kernel work formulas)."""
+stored DRAM traffic and its staleness check, per-kernel work formulas, the
+reference arm's line)."""
 import json
+import os
 
 import pytest
 
@@ -8,6 +10,7 @@ import bench
 from medusa_head_speculative_02_b200 import kernel_bench as KB
 from medusa_head_speculative_02_b200.synthetic import CONFIGS
 
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PK = {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0,
       "src": "measured"}
 
@@ -67,3 +70,23 @@ def test_rotation_copies():
     assert KB._copies(10 * KB.L2_BYTES) == 1
     assert KB._copies(KB.L2_BYTES // 4) == 12
     assert KB._copies(1) == 16
+
+
+def test_reference_arm_prints_one_valid_line():
+    """`bench.py --impl reference` (the fp64 oracle on the host cores) prints
+    one JSON line with the keys the bench contract asks of that arm."""
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--config", "tiny_f32", "--steps", "2", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == "verify steps/s"
+    assert line["value"] > 0 and line["unit"] == "steps/s" and line["higher_is_better"] is True
+    assert line["steps"] == 2 and line["warmup"] == 3 and line["n_gpus"] == 1
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "steps/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert line["config"]["workload"] == "tiny_f32"
