@@ -547,6 +547,8 @@ def run_tensor_parallel(args, cfg, world, rank, local):
     st.x["W2"] = shard_w2(st.x["W2"], world, rank)
     torch.cuda.empty_cache()
     sh = ShardedHeads(st.x["W1"], st.x["b1"], st.x["W2"], cfg.V, cfg.B, cfg.s)
+    # the step's heads call becomes this rank's slice + all-gather + merge,
+    # writing the same top-s buffers the rest of the step reads
     st.heads = lambda: sh(st.x["h"], out=(st.topk_idx, st.topk_val))
     for _ in range(args.warmup):
         st.run()
